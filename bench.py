@@ -1,0 +1,426 @@
+"""Benchmark of the HSTU layer hot path (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload training|long_history|mfalcon|academic|pr1_ref]
+
+One step = one pass of the whole path over one batch: for the default
+`training` workload, 8 HSTU layers forward (projection + SiLU, pointwise
+attention with rab buckets and causal masking, LayerNorm*U, output
+projection) then backward with fp32 gradient accumulation, on 64 jagged
+sequences with lengths U[1024, 8192], d=1024, 8 heads of 128, bf16.  Inputs
+are synthetic (seeded) and resident in HBM; with N GPUs each rank processes
+its own 64 sequences (weak scaling) and the fp32 gradients are all-reduced
+over NCCL.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hstu_sequential_transducer_b200 import workloads as W  # noqa: E402
+
+METRIC = "HSTU layer fwd+bwd tokens/s and TFLOP/s at max_len 8192; % of B200 BF16 peak"
+
+
+def pairs_allowed(lengths, num_targets=None):
+    tot = 0
+    for i, n in enumerate(lengths):
+        n = int(n)
+        m = 0 if num_targets is None else int(num_targets[i])
+        if m == 0:
+            tot += n * (n + 1) // 2
+        else:
+            h = n - m
+            tot += h * (h + 1) // 2 + m * h + m
+    return tot
+
+
+def workload_flops(w: W.Workload, backward: bool):
+    """Algorithmic flops of one step: per layer F_fwd = 10 T d^2 + 4 d sum|allowed|,
+    F_bwd = 2 F_fwd (masked pairs, padding and recompute not counted)."""
+    d, T = w.d_model, w.T
+    pairs = pairs_allowed(w.lengths, w.num_targets)
+    f_fwd = 10 * T * d * d + 4 * d * pairs
+    per_layer = f_fwd * (3 if backward else 1)
+    return per_layer * w.num_layers, pairs
+
+
+def describe(w: W.Workload):
+    return {
+        "training": "8 HSTU layers fwd+bwd, bf16, fp32 grad accumulation; 64 jagged sequences "
+                    "n~U[1024,8192]; d=1024, H=8, dh=128; causal, rab pos+time; N=8192",
+        "long_history": "4 HSTU layers fwd, bf16; 32 jagged sequences, power-law n on [256,8192]; "
+                        "d=512, H=4, dh=128; N=8192",
+        "mfalcon": "M-FALCON: 16 users x (4096 history + 1024 candidates), 3 layers fwd, "
+                   "candidates in microbatches of 256 against cached history K/V; d=512, H=4",
+        "academic": "2 HSTU layers fwd, bf16; 128 jagged sequences n~U[20,200]; d=64, H=2, dh=32",
+        "pr1_ref": "1 HSTU layer fwd, fp32; 4 sequences n~U[8,64]; d=64, H=2, dh=32",
+    }[w.name.replace("_subset", "")]
+
+
+def make_workload(name, rank):
+    if name == "training":
+        return W.training(data_seed=5 + 1000 * rank)
+    return W.WORKLOADS[name]()
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k] == "Active"})
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline (the fp64 oracle as it stands)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(w: W.Workload, budget_s: float):
+    """Times the oracle on a bounded sample of the workload: the shortest
+    sequences, as many as fit the budget (at least one).  Returns
+    (layer-tokens/s, description, threads)."""
+    from oracle import hstu_ref as R
+    plist = [R.LayerParams(p.W1, p.W2, p.rab_pos, p.rab_time, p.b1, p.b2, p.gamma, p.beta)
+             for p in w.params]
+    cfg = R.LayerConfig(w.num_heads, w.norm_N, w.num_pos_buckets, w.num_time_buckets, w.ln_eps)
+    order = np.argsort(w.lengths)
+    done_tokens, t_used, seqs = 0, 0.0, 0
+    for b in order:
+        sub = W.subset(w, [int(b)])
+        if w.name.startswith("training") and sub.T > 1024:
+            # the sample is a 1024-token prefix of a sequence
+            pref = 1024
+            sub.x, sub.timestamps, sub.dy = sub.x[:pref], sub.timestamps[:pref], sub.dy[:pref]
+            sub.seq_offsets = np.array([0, pref], np.int64)
+        t0 = time.perf_counter()
+        if w.backward:
+            R.stack_forward_backward(sub.x, sub.seq_offsets, sub.timestamps, sub.num_targets, plist,
+                                     cfg, sub.dy)
+        else:
+            R.stack_forward(sub.x, sub.seq_offsets, sub.timestamps, sub.num_targets, plist, cfg)
+        t_used += time.perf_counter() - t0
+        done_tokens += sub.T
+        seqs += 1
+        if t_used >= budget_s:
+            break
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            threads = max(i.get("num_threads", 1) for i in info)
+    except Exception:
+        pass
+    desc = (f"{seqs} sequence(s), {done_tokens} tokens, {w.num_layers} layers "
+            f"{'fwd+bwd' if w.backward else 'fwd'} (shortest first"
+            f"{'; 1024-token prefix' if w.name.startswith('training') else ''})")
+    return done_tokens * w.num_layers / t_used, desc, threads, t_used
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = make_workload(args.workload, 0)
+    for _ in range(args.warmup):
+        oracle_sample(w, 0.0)
+    vals, times = [], []
+    desc, threads = "", os.cpu_count()
+    for _ in range(args.steps):
+        v, desc, threads, t = oracle_sample(w, 0.0)
+        vals.append(v)
+        times.append(t)
+    value = float(np.median(vals))
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": float(np.median(times) * 1000), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: {describe(w)}",
+                       "sample": desc, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# Our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from hstu_sequential_transducer_b200 import build
+    from hstu_sequential_transducer_b200 import hstu as H
+    from hstu_sequential_transducer_b200 import stack as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    H.lib()
+
+    w = make_workload(args.workload, rank)
+    dw = S.DeviceWorkload.from_workload(w)
+    backward = w.backward
+    flops, pairs = workload_flops(w, backward)
+    dev = torch.device("cuda", local)
+
+    if args.workload == "mfalcon":
+        hist, cand = w.meta["history"], w.meta["candidates"]
+
+        def step():
+            S.mfalcon_score(dw, hist, cand, w.microbatch)
+    elif backward:
+        ts = S.TrainStep(dw)
+
+        def step():
+            ts.zero_grads()
+            ts.run()
+            if world > 1:
+                dist.all_reduce(ts.flat_grads)
+    else:
+        def step():
+            S.forward_stack(dw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    H.profiler_reset()
+    H.profiler_enable(True)
+    launches0 = H.launch_count()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = H.launch_count() - launches0
+    H.profiler_enable(False)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    kern = {}
+    for k, name in enumerate(H.KERNEL_NAMES):
+        n, tot = H.profiler_collect(k)
+        if n:
+            kern[name] = {"launches": n, "total_ms": tot, "avg_ms": tot / n}
+    H.profiler_reset()
+
+    tokens = w.T * w.num_layers * world
+    value = tokens / (ms / 1000.0)
+    tflops = flops * world / (ms / 1000.0) / 1e12
+    peaks, peak_src = read_peaks()
+
+    # dominant kernel and its roofline (algorithmic flops or bytes per launch)
+    d = w.d_model
+    per_launch = {
+        "attn_fwd": ("tensor", 4 * d * pairs),
+        "attn_bwd": ("tensor", 8 * d * pairs),
+        "proj_in": ("tensor", 8 * w.T * d * d),
+        "proj_out": ("tensor", 2 * w.T * d * d),
+        "proj_in_bwd": ("tensor", 16 * w.T * d * d),
+        "proj_out_bwd": ("tensor", 4 * w.T * d * d),
+        "ln_fwd": ("hbm", w.T * (6 * d + 8)),
+        "ln_bwd": ("hbm", w.T * (12 * d + 8)),
+    }
+    roof = None
+    if kern:
+        top = max((k for k in kern if k in per_launch), key=lambda k: kern[k]["total_ms"],
+                  default=None)
+        if top:
+            bound, work = per_launch[top]
+            avg_s = kern[top]["avg_ms"] / 1000.0
+            if bound == "tensor":
+                ach = work / avg_s / 1e12
+                peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+                unit = "TFLOP/s"
+            else:
+                ach = work / avg_s / 1e9
+                peak = peaks.get("hbm_gbs")
+                unit = "GB/s"
+            roof = {"kernel": top, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                    "frac": ach / peak, "traffic": None,
+                    "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
+                    "work_per_launch": work}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if backward and args.workload == "training" and not args.skip_e2e:
+        e2e = e2e_training(args, ts, dw, world, dist)
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: {describe(w)}",
+                       "global_batch": w.B * world, "tokens_per_step": w.T * world,
+                       "seq_len": int(w.lengths.max()), "max_len": 8192,
+                       "layers": w.num_layers, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "tflops": tflops, "pct_bf16_peak": tflops / peaks.get("bf16_tflops_sustained", 1400.0),
+            "roofline": roof, "kernels": kern, "gpu_launches": launches,
+            "clocks": clk, "e2e": e2e}
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        v, desc, threads, _ = oracle_sample(w, args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_training(args, ts, dw, world, dist):
+    """The same training step through the public API, with this step's inputs
+    copied from pinned host memory (x, offsets, timestamps, dY) and the
+    result (dX) read back, inside the timed region."""
+    import torch
+    w = dw.w
+    hx = torch.from_numpy(w.x).to(torch.bfloat16).pin_memory()
+    hoff = torch.from_numpy(w.seq_offsets).pin_memory()
+    hts = torch.from_numpy(w.timestamps).pin_memory()
+    hdy = torch.from_numpy(w.dy).to(torch.bfloat16).pin_memory()
+    hdx = torch.empty_like(hx).pin_memory()
+    h2d = hx.numel() * 2 + hoff.numel() * 8 + hts.numel() * 8 + hdy.numel() * 2
+    d2h = hdx.numel() * 2
+
+    def step():
+        dw.x.copy_(hx, non_blocking=True)
+        dw.offsets.copy_(hoff, non_blocking=True)
+        dw.timestamps.copy_(hts, non_blocking=True)
+        dw.dy.copy_(hdy, non_blocking=True)
+        ts.zero_grads()
+        dx = ts.run()
+        if world > 1:
+            dist.all_reduce(ts.flat_grads)
+        hdx.copy_(dx, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dw.x.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": w.T * w.num_layers * world / (ms / 1000.0), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="training", choices=list(W.WORKLOADS))
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

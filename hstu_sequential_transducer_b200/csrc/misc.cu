@@ -1,0 +1,146 @@
+// Small kernels of the HSTU path: bias-gradient column sums, the dQ
+// finalisation (fp32 accumulator times SiLU'(Pre_Q)), strided column copies
+// (M-FALCON history K/V cache) and the jagged-metadata validator.
+#include "common.cuh"
+#include "internal.h"
+
+namespace hstu {
+namespace {
+
+// out[c] += sum_r x[r][c]; CTA = 32 columns x 8 row-groups
+template <typename T>
+__global__ void colsum_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                              float* __restrict__ out) {
+  __shared__ float red[8][33];
+  const int tx = threadIdx.x % 32, ty = threadIdx.x / 32;
+  const int64_t c = (int64_t)blockIdx.x * 32 + tx;
+  float s = 0.f;
+  if (c < cols)
+    for (int64_t r = (int64_t)blockIdx.y * 8 + ty; r < rows; r += (int64_t)gridDim.y * 8)
+      s += to_f(x[r * ld + c]);
+  red[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0 && c < cols) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += red[k][tx];
+    atomicAdd(out + c, t);
+  }
+}
+
+template <typename T>
+__global__ void dq_finalize_kernel(const float* __restrict__ dq, const T* __restrict__ pre_q,
+                                   int64_t pre_stride, T* __restrict__ dpre_q, int64_t rows, int d) {
+  const int64_t n = rows * d;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / d;
+    const int c = (int)(i % d);
+    dpre_q[r * pre_stride + c] = from_f<T>(dq[i] * silu_grad_acc(to_f(pre_q[r * pre_stride + c])));
+  }
+}
+
+template <typename T>
+__global__ void copy_columns_kernel(const T* __restrict__ src, int64_t ss, T* __restrict__ dst,
+                                    int64_t ds, int64_t rows, int64_t cols) {
+  const int64_t n = rows * cols;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / cols, c = i % cols;
+    dst[r * ds + c] = src[r * ss + c];
+  }
+}
+
+__global__ void validate_seq_kernel(const int64_t* __restrict__ offs, int B, int64_t T,
+                                    const int32_t* __restrict__ nt, int max_len,
+                                    uint32_t* __restrict__ flags) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b > B) return;
+  uint32_t f = 0;
+  if (b == 0 && offs[0] != 0) f |= HSTU_FLAG_OFFSETS_START;
+  if (b == B && offs[B] != T) f |= HSTU_FLAG_OFFSETS_END;
+  if (b < B) {
+    const int64_t len = offs[b + 1] - offs[b];
+    if (len < 0) f |= HSTU_FLAG_OFFSETS_ORDER;
+    if (len > max_len) f |= HSTU_FLAG_SEQ_TOO_LONG;
+    if (nt && (nt[b] < 0 || (int64_t)nt[b] > len)) f |= HSTU_FLAG_TARGETS_RANGE;
+  }
+  if (f) atomicOr(flags, f);
+}
+
+// A token whose timestamp is below its predecessor's inside one sequence.
+// Sequences whose offsets fall outside [0, T] are skipped (already flagged).
+__global__ void validate_time_kernel(const int64_t* __restrict__ offs, int B, int64_t T,
+                                     const int64_t* __restrict__ ts, uint32_t* __restrict__ flags) {
+  for (int b = blockIdx.y; b < B; b += gridDim.y) {
+    const int64_t s = offs[b], e = offs[b + 1];
+    if (s < 0 || e > T || e - s <= 1) continue;
+    for (int64_t i = s + 1 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < e;
+         i += (int64_t)gridDim.x * blockDim.x)
+      if (ts[i] < ts[i - 1]) {
+        atomicOr(flags, HSTU_FLAG_TIME_ORDER);
+        break;
+      }
+  }
+}
+
+unsigned grid_for(int64_t n, int threads) {
+  int64_t g = (n + threads - 1) / threads;
+  if (g > 148 * 16) g = 148 * 16;
+  return (unsigned)(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+cudaError_t colsum_accumulate(int dtype, const void* x, int64_t rows, int64_t cols, int64_t ld,
+                              float* out, cudaStream_t s) {
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  dim3 grid((unsigned)((cols + 31) / 32), 1);
+  int64_t gy = (rows + 255) / 256;
+  const int64_t want = (4 * 148 + grid.x - 1) / grid.x;
+  grid.y = (unsigned)(gy < want ? (gy < 1 ? 1 : gy) : want);
+  if (dtype == HSTU_BF16)
+    colsum_kernel<bf16><<<grid, 256, 0, s>>>((const bf16*)x, rows, cols, ld, out);
+  else
+    colsum_kernel<float><<<grid, 256, 0, s>>>((const float*)x, rows, cols, ld, out);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t dq_finalize(int dtype, const float* dq, const void* pre_q, int64_t ps, void* dpre_q,
+                        int64_t T, int d, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const unsigned g = grid_for(T * d, 256);
+  if (dtype == HSTU_BF16)
+    dq_finalize_kernel<bf16><<<g, 256, 0, s>>>(dq, (const bf16*)pre_q, ps, (bf16*)dpre_q, T, d);
+  else
+    dq_finalize_kernel<float><<<g, 256, 0, s>>>(dq, (const float*)pre_q, ps, (float*)dpre_q, T, d);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t copy_columns(int dtype, const void* src, int64_t ss, void* dst, int64_t ds,
+                         int64_t rows, int64_t cols, cudaStream_t s) {
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  const unsigned g = grid_for(rows * cols, 256);
+  if (dtype == HSTU_BF16)
+    copy_columns_kernel<bf16><<<g, 256, 0, s>>>((const bf16*)src, ss, (bf16*)dst, ds, rows, cols);
+  else
+    copy_columns_kernel<float><<<g, 256, 0, s>>>((const float*)src, ss, (float*)dst, ds, rows, cols);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t validate_inputs(const int64_t* offs, int B, int64_t T, const int64_t* ts,
+                            const int32_t* nt, int max_len, uint32_t* flags, cudaStream_t s) {
+  validate_seq_kernel<<<(B + 1 + 255) / 256, 256, 0, s>>>(offs, B, T, nt, max_len, flags);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || B == 0 || ts == nullptr) return e;
+  dim3 grid(8, (unsigned)(B < 65535 ? B : 65535));
+  validate_time_kernel<<<grid, 256, 0, s>>>(offs, B, T, ts, flags);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

@@ -1,0 +1,163 @@
+"""Device-side drivers for stacks of HSTU layers (plumbing only).
+
+Moves a seeded workload to the GPU and runs it through the C ABI: a forward
+stack, a forward+backward training step, and M-FALCON scoring (history pass
+with K/V caching, then candidate microbatches against the cache).  Every
+layer step runs in libhstu.so.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+from . import hstu as H
+from .workloads import Workload
+
+
+def _t(a, dtype, device):
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(device=device, dtype=dtype)
+
+
+@dataclass
+class DeviceWorkload:
+    cfg: H.Config
+    x: torch.Tensor
+    offsets: torch.Tensor
+    timestamps: torch.Tensor
+    num_targets: Optional[torch.Tensor]
+    layers: List[H.LayerWeights]
+    dy: Optional[torch.Tensor]
+    w: Workload
+
+    @staticmethod
+    def from_workload(w: Workload, device="cuda", with_targets=True) -> "DeviceWorkload":
+        dtype_id = H.HSTU_BF16 if w.dtype == "bf16" else H.HSTU_F32
+        dt = H.torch_dtype(dtype_id)
+        cfg = H.make_config(w.d_model, w.num_heads, w.norm_N, dtype_id, w.num_pos_buckets,
+                            w.num_time_buckets, max(int(w.lengths.max(initial=1)), 1), w.ln_eps)
+        layers = []
+        for p in w.params:
+            layers.append(H.LayerWeights(
+                W1=_t(p.W1, dt, device), W2=_t(p.W2, dt, device),
+                rab_pos=_t(p.rab_pos, torch.float32, device),
+                rab_time=_t(p.rab_time, torch.float32, device),
+                b1=_t(p.b1, dt, device), b2=_t(p.b2, dt, device),
+                ln_gamma=_t(p.gamma, dt, device), ln_beta=_t(p.beta, dt, device)))
+        nt = _t(w.num_targets, torch.int32, device) if (with_targets and w.num_targets is not None) \
+            else None
+        return DeviceWorkload(cfg, _t(w.x, dt, device), _t(w.seq_offsets, torch.int64, device),
+                              _t(w.timestamps, torch.int64, device), nt, layers,
+                              _t(w.dy, dt, device), w)
+
+    @property
+    def B(self):
+        return self.offsets.numel() - 1
+
+    @property
+    def T(self):
+        return self.x.shape[0]
+
+
+def forward_stack(dw: DeviceWorkload, num_layers: Optional[int] = None, stream=None):
+    """Inference forward through the stack; returns the last layer's output."""
+    y = dw.x
+    for w in dw.layers[:num_layers]:
+        y = H.fwd(dw.cfg, w, y, dw.offsets, dw.timestamps, dw.num_targets, stream=stream)
+    return y
+
+
+class TrainStep:
+    """Buffers for a forward+backward step over the whole stack, allocated once."""
+
+    def __init__(self, dw: DeviceWorkload):
+        self.dw = dw
+        T = dw.T
+        _, saved_n = H.workspace_size(dw.cfg, dw.B, T)
+        dev = dw.x.device
+        self.saved = [torch.empty(saved_n, dtype=torch.uint8, device=dev) for _ in dw.layers]
+        self.acts = [dw.x] + [torch.empty_like(dw.x) for _ in dw.layers]
+        self.gbuf = [torch.empty_like(dw.x), torch.empty_like(dw.x)]
+        # every layer's fp32 gradients are views of one flat buffer (one
+        # all-reduce in data-parallel training)
+        names = ("W1", "W2", "b1", "b2", "ln_gamma", "ln_beta", "rab_pos", "rab_time")
+        gnames = ("dW1", "dW2", "db1", "db2", "dgamma", "dbeta", "drab_pos", "drab_time")
+        total = 0
+        for w in dw.layers:
+            for n in names:
+                t = getattr(w, n)
+                if t is not None:
+                    total += (t.numel() + 63) // 64 * 64
+        self.flat_grads = torch.zeros(max(total, 1), dtype=torch.float32, device=dev)
+        self.grads = []
+        o = 0
+        for w in dw.layers:
+            gb = H.LayerGradBufs()
+            for n, gn in zip(names, gnames):
+                t = getattr(w, n)
+                if t is not None:
+                    setattr(gb, gn, self.flat_grads[o:o + t.numel()].view(t.shape))
+                    o += (t.numel() + 63) // 64 * 64
+            self.grads.append(gb)
+
+    def zero_grads(self):
+        self.flat_grads.zero_()
+
+    def run(self, dy=None, stream=None):
+        """Forward (keeping activations) then backward from dy; returns dX."""
+        dw = self.dw
+        for i, w in enumerate(dw.layers):
+            H.fwd(dw.cfg, w, self.acts[i], dw.offsets, dw.timestamps, dw.num_targets,
+                  y=self.acts[i + 1], saved=self.saved[i], stream=stream)
+        g = dw.dy if dy is None else dy
+        for i in range(len(dw.layers) - 1, -1, -1):
+            out = self.gbuf[i % 2]
+            H.bwd(dw.cfg, dw.layers[i], self.acts[i], g, self.saved[i], dw.offsets, dw.timestamps,
+                  dw.num_targets, dx=out, grads=self.grads[i], stream=stream)
+            g = out
+        return g
+
+    @property
+    def y(self):
+        return self.acts[-1]
+
+
+def mfalcon_score(dw: DeviceWorkload, history: int, candidates: int, microbatch: int, stream=None):
+    """M-FALCON scoring of a workload whose users are `history` tokens followed
+    by `candidates` tokens: one history pass caching each layer's V|K, then the
+    candidates in microbatches against the cache.  Returns (y_hist, y_cand)
+    with candidate rows in input order."""
+    w = dw.w
+    B = w.B
+    dev = dw.x.device
+    d = w.d_model
+    n = history + candidates
+    assert np.all(w.lengths == n)
+    base = np.arange(B) * n
+    hist_rows = (base[:, None] + np.arange(history)[None, :]).reshape(-1)
+    hist_rows_t = torch.from_numpy(hist_rows).to(dev)
+    x_hist = dw.x.index_select(0, hist_rows_t)
+    ts_hist = dw.timestamps.index_select(0, hist_rows_t)
+    hist_off = torch.arange(B + 1, dtype=torch.int64, device=dev) * history
+    caches = []
+    y = x_hist
+    for lw in dw.layers:
+        kv = torch.empty(y.shape[0], 2 * d, dtype=y.dtype, device=dev)
+        y = H.fwd(dw.cfg, lw, y, hist_off, ts_hist, None, kv_out=kv, stream=stream)
+        caches.append(kv)
+    y_hist = y
+    y_cand = torch.empty(B * candidates, d, dtype=dw.x.dtype, device=dev)
+    for k0 in range(0, candidates, microbatch):
+        mb = min(microbatch, candidates - k0)
+        rows = (base[:, None] + history + k0 + np.arange(mb)[None, :]).reshape(-1)
+        rows_t = torch.from_numpy(rows).to(dev)
+        xc = dw.x.index_select(0, rows_t)
+        tc = dw.timestamps.index_select(0, rows_t)
+        coff = torch.arange(B + 1, dtype=torch.int64, device=dev) * mb
+        for li, lw in enumerate(dw.layers):
+            xc = H.fwd_cached(dw.cfg, lw, xc, coff, tc, caches[li], hist_off, ts_hist, stream=stream)
+        out_rows = (np.arange(B)[:, None] * candidates + k0 + np.arange(mb)[None, :]).reshape(-1)
+        y_cand[torch.from_numpy(out_rows).to(dev)] = xc
+    return y_hist, y_cand

@@ -28,21 +28,43 @@ from __future__ import annotations
 from dataclasses import dataclass, field
 from typing import Dict, List, Optional
 
+import os
+
 import numpy as np
 
 
 def round_to_bf16(a) -> np.ndarray:
     """Round float32 values to the nearest bf16 value (ties to even) and
-    return them as float32 (exactly representable in bf16)."""
+    return them as float32 (exactly representable in bf16).  Uses torch's
+    CPU conversion, which rounds to nearest even."""
+    import torch
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> np.uint64(16)) & np.uint64(1)
-    u = (u + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)
-    out = u.astype(np.uint32).view(np.float32)
-    nan = np.isnan(a)
-    if nan.any():
-        out = out.copy()
-        out[nan] = np.nan
+    return torch.from_numpy(a).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def normal_rows(seed: int, rows: int, cols: int, bf16: bool, std: float = 1.0,
+                chunk: int = 8192) -> np.ndarray:
+    """N(0, std^2) float32 matrix [rows, cols]; row-chunk k is drawn from the
+    k-th child of SeedSequence(seed), so chunks fill in parallel threads and
+    the result does not depend on the thread count."""
+    import concurrent.futures as cf
+    import torch
+    out = np.empty((rows, cols), dtype=np.float32)
+    nchunks = (rows + chunk - 1) // chunk
+    children = np.random.SeedSequence(seed).spawn(max(nchunks, 1))
+
+    def fill(k):
+        r0, r1 = k * chunk, min(rows, (k + 1) * chunk)
+        blk = out[r0:r1]
+        np.random.default_rng(children[k]).standard_normal(size=blk.shape, dtype=np.float32, out=blk)
+        if std != 1.0:
+            blk *= np.float32(std)
+        if bf16:
+            t = torch.from_numpy(blk)
+            t.copy_(t.to(torch.bfloat16).to(torch.float32))
+
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 4)) as ex:
+        list(ex.map(fill, range(nchunks)))
     return out
 
 
@@ -170,8 +192,8 @@ def _finish(name, dtype, d, H, N, layers, lengths, rng, seed, x=None, num_target
     if timestamps is None:
         timestamps = draw_timestamps(rng, lengths)
     if x is None:
-        x = rng.normal(0.0, 1.0, size=(T, d)).astype(np.float32)
-    if bf16:
+        x = normal_rows(int(rng.integers(0, 2**62)), T, d, bf16)
+    elif bf16:
         x = round_to_bf16(x)
     params = []
     for layer in range(layers):
@@ -180,10 +202,7 @@ def _finish(name, dtype, d, H, N, layers, lengths, rng, seed, x=None, num_target
                                   with_affine=with_affine))
     dy = None
     if backward:
-        grng = np.random.default_rng(seed * 1000 + 999)
-        dy = grng.normal(0.0, 1.0, size=(T, d)).astype(np.float32)
-        if bf16:
-            dy = round_to_bf16(dy)
+        dy = normal_rows(seed * 1000 + 999, T, d, bf16)
     return Workload(name=name, dtype=dtype, d_model=d, num_heads=H, norm_N=float(N),
                     num_layers=layers, x=x, seq_offsets=offs, timestamps=timestamps,
                     num_targets=num_targets, params=params, dy=dy, backward=backward,
@@ -233,10 +252,15 @@ def mfalcon(seed: int = 4, users: int = 16, history: int = 4096, candidates: int
                    meta={"history": history, "candidates": candidates})
 
 
-def training(seed: int = 5, B: int = 64) -> Workload:
-    rng = np.random.default_rng(seed)
+def training(seed: int = 5, B: int = 64, data_seed: Optional[int] = None) -> Workload:
+    """`data_seed` (default: seed) draws lengths, inputs and timestamps;
+    weights always come from `seed`, so data-parallel ranks share them."""
+    rng = np.random.default_rng(seed if data_seed is None else data_seed)
     lengths = rng.integers(1024, 8193, size=B)
-    return _finish("training", "bf16", 1024, 8, 8192, 8, lengths, rng, seed, backward=True)
+    w = _finish("training", "bf16", 1024, 8, 8192, 8, lengths, rng, seed, backward=True)
+    if data_seed is not None and data_seed != seed:
+        w.dy = normal_rows(data_seed * 1000 + 999, w.T, w.d_model, True)
+    return w
 
 
 WORKLOADS = {
@@ -255,7 +279,7 @@ def custom(lengths, d=64, H=2, N=64.0, dtype="f32", layers=1, seed=11, num_targe
     rng = np.random.default_rng(seed)
     lengths = np.asarray(lengths, dtype=np.int64)
     T = int(lengths.sum())
-    x = (rng.normal(0.0, x_std, size=(T, d))).astype(np.float32)
+    x = normal_rows(int(rng.integers(0, 2**62)), T, d, False, std=x_std)
     if timestamps is None:
         timestamps = draw_timestamps(rng, lengths, mean_gap=mean_gap)
     nt = None if num_targets is None else np.asarray(num_targets, dtype=np.int32)

@@ -467,3 +467,114 @@ def layer_flops_fwd(lengths, num_targets, d: int) -> int:
                 for n, m in zip(lengths, num_targets if num_targets is not None
                                 else [0] * len(lengths)))
     return 10 * T * d * d + 4 * d * pairs
+
+
+# ----------------------------------------------------------------------------
+# Single steps of the layer (for per-kernel parity).  Each restates one
+# equation on jagged inputs; the CPU tests check that they compose back into
+# layer_forward / layer_backward above.
+# ----------------------------------------------------------------------------
+
+def attention_forward(g, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
+                      cfg: LayerConfig):
+    """Equation (2) alone: O[T, d] from G = U|V|Q|K [T, 4d]."""
+    g = np.asarray(g, dtype=F64)
+    T, d4 = g.shape
+    d = d4 // 4
+    H = cfg.num_heads
+    dh = d // H
+    offs = np.asarray(seq_offsets, dtype=np.int64)
+    ts = np.asarray(timestamps, dtype=np.int64)
+    o = np.zeros((T, d))
+    for b in range(len(offs) - 1):
+        s, e = int(offs[b]), int(offs[b + 1])
+        n = e - s
+        m = 0 if num_targets is None else int(num_targets[b])
+        mask = allowed_mask(n, m)
+        _, V, Q, K = _split(g[s:e], d)
+        for hh in range(H):
+            cs = slice(hh * dh, (hh + 1) * dh)
+            bias = rab_bias(n, m, ts[s:e],
+                            None if rab_pos is None else rab_pos[hh],
+                            None if rab_time is None else rab_time[hh],
+                            cfg.num_pos_buckets, cfg.num_time_buckets)
+            S = Q[:, cs] @ K[:, cs].T + bias
+            o[s:e, cs] = (np.where(mask, silu(S), 0.0) / cfg.norm_N) @ V[:, cs]
+    return o
+
+
+def ln_gate_forward(o, u, gamma, beta, eps):
+    """Z = (LayerNorm(O) * gamma + beta) * U over each row; returns z, mean, rstd."""
+    o = np.asarray(o, dtype=F64)
+    mu = o.mean(axis=1, keepdims=True)
+    var = ((o - mu) ** 2).mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + eps)
+    ln = (o - mu) * rstd
+    if gamma is not None:
+        ln = ln * np.asarray(gamma, F64)
+    if beta is not None:
+        ln = ln + np.asarray(beta, F64)
+    return ln * np.asarray(u, F64), mu[:, 0], rstd[:, 0]
+
+
+def attention_backward(g, do, seq_offsets, timestamps, num_targets, rab_pos, rab_time,
+                       cfg: LayerConfig):
+    """Backward of attention_forward: returns dG [T, 4d] (U block zero),
+    drab_pos [H, P], drab_time [H, Bt]."""
+    g = np.asarray(g, dtype=F64)
+    do = np.asarray(do, dtype=F64)
+    T, d4 = g.shape
+    d = d4 // 4
+    H = cfg.num_heads
+    dh = d // H
+    P, Bt = cfg.num_pos_buckets, cfg.num_time_buckets
+    offs = np.asarray(seq_offsets, dtype=np.int64)
+    ts = np.asarray(timestamps, dtype=np.int64)
+    dg = np.zeros((T, 4 * d))
+    drp = np.zeros((H, P))
+    drt = np.zeros((H, Bt))
+    for b in range(len(offs) - 1):
+        s, e = int(offs[b]), int(offs[b + 1])
+        n = e - s
+        m = 0 if num_targets is None else int(num_targets[b])
+        mask = allowed_mask(n, m)
+        bp, bt = bucket_ids(n, m, ts[s:e], P, Bt)
+        _, V, Q, K = _split(g[s:e], d)
+        for hh in range(H):
+            cs = slice(hh * dh, (hh + 1) * dh)
+            bias = np.zeros((n, n))
+            if rab_pos is not None:
+                bias = bias + np.asarray(rab_pos[hh], F64)[bp]
+            if rab_time is not None:
+                bias = bias + np.asarray(rab_time[hh], F64)[bt]
+            S = Q[:, cs] @ K[:, cs].T + bias
+            A = np.where(mask, silu(S), 0.0) / cfg.norm_N
+            dA = do[s:e, cs] @ V[:, cs].T
+            dS = np.where(mask, dA * silu_grad(S), 0.0) / cfg.norm_N
+            dg[s:e, d + hh * dh:d + (hh + 1) * dh] = A.T @ do[s:e, cs]
+            dg[s:e, 2 * d + hh * dh:2 * d + (hh + 1) * dh] = dS @ K[:, cs]
+            dg[s:e, 3 * d + hh * dh:3 * d + (hh + 1) * dh] = dS.T @ Q[:, cs]
+            np.add.at(drp[hh], bp[mask], dS[mask])
+            np.add.at(drt[hh], bt[mask], dS[mask])
+    return dg, drp, drt
+
+
+def ln_gate_backward(dz, o, u, gamma, beta, eps):
+    """Backward of ln_gate_forward: returns do, du, dgamma, dbeta."""
+    dz = np.asarray(dz, F64)
+    o = np.asarray(o, F64)
+    u = np.asarray(u, F64)
+    d = o.shape[1]
+    gm = np.ones(d) if gamma is None else np.asarray(gamma, F64)
+    bt = np.zeros(d) if beta is None else np.asarray(beta, F64)
+    mu = o.mean(axis=1, keepdims=True)
+    var = ((o - mu) ** 2).mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + eps)
+    ohat = (o - mu) * rstd
+    ln = ohat * gm + bt
+    dln = dz * u
+    du = dz * ln
+    dohat = dln * gm
+    do = rstd * (dohat - dohat.mean(axis=1, keepdims=True)
+                 - ohat * (dohat * ohat).mean(axis=1, keepdims=True))
+    return do, du, (dln * ohat).sum(axis=0), dln.sum(axis=0)

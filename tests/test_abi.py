@@ -1,0 +1,94 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects
+host-checkable errors before touching the GPU (CPU only; no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hstu_sequential_transducer_b200 import build
+from hstu_sequential_transducer_b200 import hstu as H
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return H.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "hstu.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hstu_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(L, n), n
+    # and the binding covers every one of them
+    assert set(names) <= set(H.exported_symbols())
+
+
+def test_status_strings(L):
+    assert H.status_string(0) == "ok"
+    assert "workspace" in H.status_string(4)
+    assert H.version().startswith("hstu-b200")
+
+
+def cfg(**kw):
+    c = H.make_config(kw.pop("d", 64), kw.pop("H", 2), kw.pop("N", 64.0), kw.pop("dtype", H.HSTU_BF16))
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def test_config_validation(L):
+    ws, sv = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    call = lambda c: L.hstu_workspace_size(ctypes.byref(c) if c is not None else None, 4, 100,
+                                           ctypes.byref(ws), ctypes.byref(sv))
+    assert call(None) == 1
+    assert call(cfg()) == 0 and ws.value > 0 and sv.value > 0
+    assert call(cfg(head_dim=48, d_model=96)) == 2           # dh not built
+    assert call(cfg(d_model=65, head_dim=65, num_heads=1)) == 2      # dh not built
+    assert call(cfg(num_heads=3)) == 1                         # d != H * dh
+    assert call(cfg(norm_N=0.0)) == 1
+    assert call(cfg(num_pos_buckets=33)) == 2
+    assert call(cfg(dtype=7)) == 1
+    assert L.hstu_workspace_size(ctypes.byref(cfg()), -1, 10, None, None) == 1
+
+
+def test_saved_layout_sizes(L):
+    c = cfg(d=1024, H=8)
+    off = H.saved_layout(c, 1000)
+    d, es = 1024, 2
+    assert off[1] - off[0] >= 1000 * 4 * d * es
+    assert off[3] - off[2] >= 1000 * d * es
+    assert off[6] >= off[5] + 1000 * 4
+    assert all(o % 256 == 0 for o in off)
+
+
+def test_host_argument_errors_return_before_launch(L):
+    c = cfg()
+    w = H.Weights(None, None, None, None, None, None, None, None)
+    # null x with T > 0
+    assert L.hstu_proj_in_fwd(ctypes.byref(c), ctypes.byref(w), None, 10, None, None, None) == 1
+    # misaligned pointer -> unsupported
+    w.W1 = 0x1000
+    assert L.hstu_proj_in_fwd(ctypes.byref(c), ctypes.byref(w), 0x2001, 10, None, 0x3000, None) == 2
+    # workspace too small for the layer forward
+    off = (ctypes.c_int64 * 3)()
+    w.W2 = 0x1000
+    st = L.hstu_fwd(ctypes.byref(c), ctypes.byref(w), 0x2000, ctypes.addressof(off), 2, 10,
+                    0x4000, None, 0x5000, None, None, 0x6000, 16, None)
+    assert st == 4
+    # empty input is a no-op success (no launch)
+    st = L.hstu_fwd(ctypes.byref(c), ctypes.byref(w), None, ctypes.addressof(off), 0, 0, None, None,
+                    None, None, None, None, 1 << 30, None)
+    assert st == 0
+    # negative sizes
+    assert L.hstu_ln_gate_fwd(ctypes.byref(c), None, None, None, None, -1, None, None, None,
+                              None) == 1

@@ -1,0 +1,490 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Tolerance (stated per dtype, on the compared tensor):
+    max |gpu - oracle| <= 1e-4 * rms(oracle)   for fp32
+    max |gpu - oracle| <= 2e-2 * rms(oracle)   for bf16
+The oracle consumes the exact (bf16-rounded) inputs the GPU sees, in fp64.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hstu_ref as R
+from hstu_sequential_transducer_b200 import build
+from hstu_sequential_transducer_b200 import hstu as H
+from hstu_sequential_transducer_b200 import stack as S
+from hstu_sequential_transducer_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    H.lib()
+
+
+def rel_err(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), "non-finite values from the GPU"
+    rms = np.sqrt(np.mean(ref ** 2)) if ref.size else 1.0
+    return float(np.max(np.abs(got - ref)) / max(rms, 1e-30)) if ref.size else 0.0
+
+
+def check(got, ref, dtype, what, scale=1.0):
+    e = rel_err(got, ref)
+    assert e <= TOL[dtype] * scale, f"{what}: max|err|/rms = {e:.3e} > {TOL[dtype] * scale:.1e}"
+    return e
+
+
+def np_(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def lp(p: W.Params) -> R.LayerParams:
+    return R.LayerParams(p.W1, p.W2, p.rab_pos, p.rab_time, p.b1, p.b2, p.gamma, p.beta)
+
+
+def lcfg(w: W.Workload) -> R.LayerConfig:
+    return R.LayerConfig(w.num_heads, w.norm_N, w.num_pos_buckets, w.num_time_buckets, w.ln_eps)
+
+
+def dev_rows(a, dtype):
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(DEV, dt)
+
+
+def rand_g(rng, T, d, dtype, scale=1.0):
+    """A random U|V|Q|K block (post-SiLU-like, values in a bf16-friendly range)."""
+    g = (rng.normal(0.0, scale, size=(T, 4 * d))).astype(np.float32)
+    return W.round_to_bf16(g) if dtype == "bf16" else g
+
+
+RAGGED = [300, 1, 0, 129, 64, 65, 257]
+
+
+# ----------------------------------------------------------------------------
+# Single steps
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d,Hh", [(64, 2), (256, 2), (512, 4)])
+def test_proj_in_parity(dtype, d, Hh):
+    w = W.custom([200, 77, 1, 0, 300], d=d, H=Hh, dtype=dtype, with_bias=True)
+    dw = S.DeviceWorkload.from_workload(w)
+    T = w.T
+    pre = torch.empty(T, 4 * d, dtype=dw.x.dtype, device=DEV)
+    g = torch.empty_like(pre)
+    H.proj_in_fwd(dw.cfg, dw.layers[0], dw.x, pre, g)
+    p = lp(w.params[0]).as_f64()
+    ref_pre = w.x.astype(np.float64) @ p.W1 + p.b1
+    check(np_(pre), ref_pre, dtype, "Pre")
+    check(np_(g), R.silu(ref_pre), dtype, "G")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dh", [32, 64, 128])
+@pytest.mark.parametrize("targets", [False, True])
+def test_attention_fwd_parity(dtype, dh, targets):
+    Hh = 2
+    d = Hh * dh
+    lengths = RAGGED
+    nt = [40, 1, 0, 129, 0, 7, 100] if targets else None
+    w = W.custom(lengths, d=d, H=Hh, dtype=dtype, N=300.0, num_targets=nt, mean_gap=3000.0)
+    rng = np.random.default_rng(dh)
+    g = rand_g(rng, w.T, d, dtype, scale=0.5)
+    dw = S.DeviceWorkload.from_workload(w)
+    gd = dev_rows(g, dtype)
+    o = torch.empty(w.T, d, dtype=gd.dtype, device=DEV)
+    p = w.params[0]
+    H.attention_fwd(dw.cfg, dw.layers[0].rab_pos, dw.layers[0].rab_time, gd, dw.offsets,
+                    dw.timestamps, dw.num_targets, o)
+    ref = R.attention_forward(g, w.seq_offsets, w.timestamps, w.num_targets, p.rab_pos,
+                              p.rab_time, lcfg(w))
+    check(np_(o), ref, dtype, "O")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 512, 1024])
+def test_ln_gate_fwd_parity(dtype, d):
+    w = W.custom([100, 33, 0, 9], d=d, H=d // 64 if d >= 64 else 1, dtype=dtype, with_affine=True)
+    rng = np.random.default_rng(1)
+    o = rng.normal(0, 0.3, size=(w.T, d)).astype(np.float32)
+    g = rand_g(rng, w.T, d, dtype)
+    if dtype == "bf16":
+        o = W.round_to_bf16(o)
+    dw = S.DeviceWorkload.from_workload(w)
+    z = torch.empty(w.T, d, dtype=dw.x.dtype, device=DEV)
+    mean = torch.empty(w.T, dtype=torch.float32, device=DEV)
+    rstd = torch.empty_like(mean)
+    H.ln_gate_fwd(dw.cfg, dw.layers[0].ln_gamma, dw.layers[0].ln_beta, dev_rows(o, dtype),
+                  dev_rows(g, dtype), z, mean, rstd)
+    p = w.params[0]
+    rz, rmu, rrs = R.ln_gate_forward(o, g[:, :d], p.gamma, p.beta, w.ln_eps)
+    check(np_(z), rz, dtype, "Z")
+    check(np_(mean), rmu, "f32", "mean", scale=10)
+    np.testing.assert_allclose(np_(rstd), rrs, rtol=1e-4)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_proj_out_parity(dtype):
+    d = 256
+    w = W.custom([150, 0, 81], d=d, H=2, dtype=dtype, with_bias=True)
+    rng = np.random.default_rng(2)
+    z = rng.normal(0, 1, size=(w.T, d)).astype(np.float32)
+    if dtype == "bf16":
+        z = W.round_to_bf16(z)
+    dw = S.DeviceWorkload.from_workload(w)
+    y = torch.empty(w.T, d, dtype=dw.x.dtype, device=DEV)
+    H.proj_out_fwd(dw.cfg, dw.layers[0].W2, dw.layers[0].b2, dev_rows(z, dtype), dw.x, y)
+    p = lp(w.params[0]).as_f64()
+    ref = z.astype(np.float64) @ p.W2 + p.b2 + w.x
+    check(np_(y), ref, dtype, "Y")
+
+
+# ----------------------------------------------------------------------------
+# Backward steps
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_proj_out_bwd_parity(dtype):
+    d = 128
+    w = W.custom([150, 0, 81, 300], d=d, H=2, dtype=dtype, with_bias=True, backward=True)
+    rng = np.random.default_rng(3)
+    z = rng.normal(0, 1, size=(w.T, d)).astype(np.float32)
+    if dtype == "bf16":
+        z = W.round_to_bf16(z)
+    dw = S.DeviceWorkload.from_workload(w)
+    dz = torch.empty(w.T, d, dtype=dw.x.dtype, device=DEV)
+    dW2 = torch.zeros(d, d, dtype=torch.float32, device=DEV)
+    db2 = torch.zeros(d, dtype=torch.float32, device=DEV)
+    H.proj_out_bwd(dw.cfg, dw.layers[0].W2, dev_rows(z, dtype), dw.dy, dz, dW2, db2)
+    p = lp(w.params[0]).as_f64()
+    dy = w.dy.astype(np.float64)
+    check(np_(dz), dy @ p.W2.T, dtype, "dZ")
+    check(np_(dW2), z.astype(np.float64).T @ dy, dtype, "dW2")
+    check(np_(db2), dy.sum(0), dtype, "db2")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 1024])
+def test_ln_gate_bwd_parity(dtype, d):
+    w = W.custom([100, 33, 0, 9], d=d, H=max(1, d // 128), dtype=dtype, with_affine=True)
+    rng = np.random.default_rng(4)
+    o = rng.normal(0, 0.3, size=(w.T, d)).astype(np.float32)
+    dz = rng.normal(0, 1, size=(w.T, d)).astype(np.float32)
+    pre = rng.normal(0, 1, size=(w.T, 4 * d)).astype(np.float32)
+    if dtype == "bf16":
+        o, dz, pre = W.round_to_bf16(o), W.round_to_bf16(dz), W.round_to_bf16(pre)
+    g = R.silu(pre.astype(np.float64)).astype(np.float32)
+    if dtype == "bf16":
+        g = W.round_to_bf16(g)
+    dw = S.DeviceWorkload.from_workload(w)
+    lw = dw.layers[0]
+    p = w.params[0]
+    _, mu, rs = R.ln_gate_forward(o, g[:, :d], p.gamma, p.beta, w.ln_eps)
+    dO = torch.empty(w.T, d, dtype=dw.x.dtype, device=DEV)
+    dpre = torch.zeros(w.T, 4 * d, dtype=dw.x.dtype, device=DEV)
+    dgam = torch.zeros(d, dtype=torch.float32, device=DEV)
+    dbet = torch.zeros(d, dtype=torch.float32, device=DEV)
+    H.ln_gate_bwd(dw.cfg, lw.ln_gamma, lw.ln_beta, dev_rows(dz, dtype), dev_rows(o, dtype),
+                  dev_rows(g, dtype), dev_rows(pre, dtype),
+                  torch.tensor(mu, dtype=torch.float32, device=DEV),
+                  torch.tensor(rs, dtype=torch.float32, device=DEV), dO, dpre, dgam, dbet)
+    rdo, rdu, rdg, rdb = R.ln_gate_backward(dz, o, g[:, :d], p.gamma, p.beta, w.ln_eps)
+    check(np_(dO), rdo, dtype, "dO")
+    check(np_(dpre)[:, :d], rdu * R.silu_grad(pre[:, :d].astype(np.float64)), dtype, "dPre_U")
+    check(np_(dgam), rdg, dtype, "dgamma")
+    check(np_(dbet), rdb, dtype, "dbeta")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dh", [32, 128])
+@pytest.mark.parametrize("targets", [False, True])
+def test_attention_bwd_parity(dtype, dh, targets):
+    Hh = 2
+    d = Hh * dh
+    nt = [40, 1, 0, 129, 0, 7, 100] if targets else None
+    w = W.custom(RAGGED, d=d, H=Hh, dtype=dtype, N=300.0, num_targets=nt, mean_gap=3000.0)
+    rng = np.random.default_rng(10 + dh)
+    pre = rng.normal(0, 1, size=(w.T, 4 * d)).astype(np.float32)
+    if dtype == "bf16":
+        pre = W.round_to_bf16(pre)
+    g = R.silu(pre.astype(np.float64)).astype(np.float32)
+    if dtype == "bf16":
+        g = W.round_to_bf16(g)
+    dout = rng.normal(0, 1, size=(w.T, d)).astype(np.float32)
+    if dtype == "bf16":
+        dout = W.round_to_bf16(dout)
+    dw = S.DeviceWorkload.from_workload(w)
+    lw = dw.layers[0]
+    dpre = torch.zeros(w.T, 4 * d, dtype=dw.x.dtype, device=DEV)
+    drp = torch.zeros_like(lw.rab_pos)
+    drt = torch.zeros_like(lw.rab_time)
+    H.attention_bwd(dw.cfg, lw.rab_pos, lw.rab_time, dev_rows(g, dtype), dev_rows(pre, dtype),
+                    dev_rows(dout, dtype), dw.offsets, dw.timestamps, dw.num_targets, dpre, drp, drt)
+    p = w.params[0]
+    dg, rdp, rdt = R.attention_backward(g, dout, w.seq_offsets, w.timestamps, w.num_targets,
+                                        p.rab_pos, p.rab_time, lcfg(w))
+    sg = R.silu_grad(pre.astype(np.float64))
+    got = np_(dpre)
+    for name, sl in (("dPre_V", slice(d, 2 * d)), ("dPre_Q", slice(2 * d, 3 * d)),
+                     ("dPre_K", slice(3 * d, 4 * d))):
+        check(got[:, sl], dg[:, sl] * sg[:, sl], dtype, name)
+    check(np_(drp), rdp, dtype, "drab_pos")
+    check(np_(drt), rdt, dtype, "drab_time")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_proj_in_bwd_parity(dtype):
+    d = 128
+    w = W.custom([150, 0, 81, 300], d=d, H=2, dtype=dtype, with_bias=True, backward=True)
+    rng = np.random.default_rng(5)
+    dpre = rng.normal(0, 1, size=(w.T, 4 * d)).astype(np.float32)
+    if dtype == "bf16":
+        dpre = W.round_to_bf16(dpre)
+    dw = S.DeviceWorkload.from_workload(w)
+    dx = torch.empty(w.T, d, dtype=dw.x.dtype, device=DEV)
+    dW1 = torch.zeros(d, 4 * d, dtype=torch.float32, device=DEV)
+    db1 = torch.zeros(4 * d, dtype=torch.float32, device=DEV)
+    H.proj_in_bwd(dw.cfg, dw.layers[0].W1, dw.x, dev_rows(dpre, dtype), dw.dy, dx, dW1, db1)
+    p = lp(w.params[0]).as_f64()
+    dp = dpre.astype(np.float64)
+    check(np_(dx), dp @ p.W1.T + w.dy, dtype, "dX")
+    check(np_(dW1), w.x.astype(np.float64).T @ dp, dtype, "dW1")
+    check(np_(db1), dp.sum(0), dtype, "db1")
+
+
+# ----------------------------------------------------------------------------
+# Whole layers and stacks
+# ----------------------------------------------------------------------------
+
+def oracle_stack(w: W.Workload):
+    return R.stack_forward(w.x, w.seq_offsets, w.timestamps, w.num_targets,
+                           [lp(p) for p in w.params], lcfg(w))
+
+
+def test_pr1_ref_layer_fp32():
+    w = W.pr1_ref()
+    dw = S.DeviceWorkload.from_workload(w)
+    y = S.forward_stack(dw)
+    check(np_(y), oracle_stack(w), "f32", "Y pr1_ref")
+
+
+def test_academic_stack_bf16():
+    w = W.academic()
+    dw = S.DeviceWorkload.from_workload(w)
+    y = S.forward_stack(dw)
+    ref = oracle_stack(w)
+    check(np_(y), ref, "bf16", "Y academic")
+    # the residual dominates Y; the branch alone is held to the same bound
+    check(np_(y) - w.x, ref - w.x, "bf16", "Y - X academic", scale=2.5)
+
+
+def test_long_history_subset_bf16():
+    w = W.long_history()
+    order = np.argsort(w.lengths)
+    sub = W.subset(w, sorted(order[:3].tolist()) + [int(order[-1])])
+    dw = S.DeviceWorkload.from_workload(sub)
+    y = np_(S.forward_stack(dw))
+    # short sequences whole; the longest one on its first 384 tokens (causal prefix)
+    keep = sorted(order[:3].tolist())
+    small = W.subset(w, keep)
+    ref_small = oracle_stack(small)
+    n_small = small.T
+    check(y[:n_small], ref_small, "bf16", "Y long_history short seqs")
+    longest = W.subset(w, [int(order[-1])])
+    pref = 384
+    longest.x, longest.timestamps = longest.x[:pref], longest.timestamps[:pref]
+    longest.seq_offsets = np.array([0, pref], np.int64)
+    check(y[n_small:n_small + pref], oracle_stack(longest), "bf16", "Y long_history prefix")
+
+
+def test_layer_fwd_bwd_parity_small():
+    for dtype in ("f32", "bf16"):
+        w = W.custom([70, 1, 0, 130, 33], d=128, H=2, dtype=dtype, N=120.0, num_targets=[5, 0, 0, 20, 33],
+                     with_bias=True, with_affine=True, backward=True, layers=2, mean_gap=900.0)
+        dw = S.DeviceWorkload.from_workload(w)
+        step = S.TrainStep(dw)
+        step.zero_grads()
+        dx = step.run()
+        torch.cuda.synchronize()
+        y, rdx, rgr = R.stack_forward_backward(w.x, w.seq_offsets, w.timestamps, w.num_targets,
+                                               [lp(p) for p in w.params], lcfg(w), w.dy)
+        check(np_(step.y), y, dtype, f"Y {dtype}")
+        check(np_(dx), rdx, dtype, f"dX {dtype}")
+        for li in range(2):
+            g = step.grads[li]
+            for name, got, ref in (("dW1", g.dW1, rgr[li].dW1), ("dW2", g.dW2, rgr[li].dW2),
+                                   ("db1", g.db1, rgr[li].db1), ("db2", g.db2, rgr[li].db2),
+                                   ("dgamma", g.dgamma, rgr[li].dgamma),
+                                   ("dbeta", g.dbeta, rgr[li].dbeta),
+                                   ("drab_pos", g.drab_pos, rgr[li].drab_pos),
+                                   ("drab_time", g.drab_time, rgr[li].drab_time)):
+                check(np_(got), ref, dtype, f"layer {li} {name} {dtype}")
+
+
+@pytest.fixture(scope="module")
+def training_oracle():
+    """fp64 oracle of the 8-layer training workload on its two shortest
+    sequences (forward, backward from the workload's dY, all gradients)."""
+    w = W.training()
+    order = np.argsort(w.lengths)
+    seqs = sorted(order[:2].tolist())
+    sub = W.subset(w, seqs)
+    y, rdx, rgr = R.stack_forward_backward(sub.x, sub.seq_offsets, sub.timestamps, None,
+                                           [lp(p) for p in sub.params], lcfg(sub), sub.dy)
+    return w, seqs, sub, y, rdx, rgr
+
+
+def test_training_subset_fwd_bwd_bf16(training_oracle):
+    """The 8-layer training workload restricted to its two shortest
+    sequences: every output and gradient against the oracle."""
+    w, seqs, sub, y, rdx, rgr = training_oracle
+    dw = S.DeviceWorkload.from_workload(sub)
+    step = S.TrainStep(dw)
+    step.zero_grads()
+    dx = step.run()
+    torch.cuda.synchronize()
+    check(np_(step.y), y, "bf16", "Y training subset")
+    check(np_(dx), rdx, "bf16", "dX training subset")
+    for li in range(8):
+        g = step.grads[li]
+        for name, got, ref in (("dW1", g.dW1, rgr[li].dW1), ("dW2", g.dW2, rgr[li].dW2),
+                               ("dgamma", g.dgamma, rgr[li].dgamma),
+                               ("dbeta", g.dbeta, rgr[li].dbeta),
+                               ("drab_pos", g.drab_pos, rgr[li].drab_pos),
+                               ("drab_time", g.drab_time, rgr[li].drab_time)):
+            check(np_(got), ref, "bf16", f"layer {li} {name}")
+
+
+def test_training_full_size_sampled(training_oracle):
+    """The full training workload (64 sequences, 8 layers, fwd+bwd) in the
+    launch configuration the benchmark times; Y and dX rows of the two sampled
+    sequences against the oracle (sequences are independent in Y and dX)."""
+    w, seqs, sub, y, rdx, rgr = training_oracle
+    dw = S.DeviceWorkload.from_workload(w)
+    step = S.TrainStep(dw)
+    step.zero_grads()
+    dx = step.run()
+    torch.cuda.synchronize()
+    rows = np.concatenate([np.arange(w.seq_offsets[b], w.seq_offsets[b + 1]) for b in seqs])
+    rows_t = torch.from_numpy(rows).cuda()
+    check(np_(step.y.index_select(0, rows_t)), y, "bf16", "Y full-size sampled")
+    check(np_(dx.index_select(0, rows_t)), rdx, "bf16", "dX full-size sampled")
+    # every gradient finite and non-trivial at full size
+    for g in step.grads:
+        for t in (g.dW1, g.dW2, g.drab_pos, g.drab_time):
+            a = t.float()
+            assert torch.isfinite(a).all() and a.abs().max() > 0
+
+
+# ----------------------------------------------------------------------------
+# M-FALCON
+# ----------------------------------------------------------------------------
+
+def small_mfalcon(users=2, history=300, candidates=70):
+    return W.mfalcon(seed=8, users=users, history=history, candidates=candidates, microbatch=32)
+
+
+def test_mfalcon_target_mask_full_sequence_parity():
+    w = small_mfalcon()
+    dw = S.DeviceWorkload.from_workload(w)
+    y = S.forward_stack(dw)
+    check(np_(y), oracle_stack(w), "bf16", "Y mfalcon full-sequence")
+
+
+@pytest.mark.parametrize("mb", [1, 32, 70])
+def test_mfalcon_cached_microbatches(mb):
+    w = small_mfalcon()
+    dw = S.DeviceWorkload.from_workload(w)
+    y_hist, y_cand = S.mfalcon_score(dw, 300, 70, mb)
+    ref = oracle_stack(w)
+    n = 370
+    hist_rows = np.concatenate([np.arange(b * n, b * n + 300) for b in range(2)])
+    cand_rows = np.concatenate([np.arange(b * n + 300, (b + 1) * n) for b in range(2)])
+    check(np_(y_hist), ref[hist_rows], "bf16", "Y history (cached pass)")
+    check(np_(y_cand), ref[cand_rows], "bf16", f"Y candidates mb={mb}")
+
+
+def test_mfalcon_cached_matches_gpu_full_sequence():
+    """Candidate scores do not depend on the microbatch split (GPU vs GPU)."""
+    w = small_mfalcon()
+    dw = S.DeviceWorkload.from_workload(w)
+    y_full = np_(S.forward_stack(dw))
+    _, c1 = S.mfalcon_score(dw, 300, 70, 1)
+    _, c70 = S.mfalcon_score(dw, 300, 70, 70)
+    cand_rows = np.concatenate([np.arange(b * 370 + 300, (b + 1) * 370) for b in range(2)])
+    check(np_(c1), np_(c70), "bf16", "mb=1 vs mb=70", scale=0.5)
+    check(np_(c70), y_full[cand_rows], "bf16", "cached vs full-sequence", scale=0.5)
+
+
+# ----------------------------------------------------------------------------
+# Edge cases
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_edge_lengths_and_all_candidates(dtype):
+    lengths = [0, 1, 0, 2, 127, 128, 129, 1, 3]
+    nt = [0, 1, 0, 2, 0, 128, 1, 0, 3]      # includes all-candidate sequences
+    w = W.custom(lengths, d=64, H=2, dtype=dtype, N=64.0, num_targets=nt, with_affine=True)
+    dw = S.DeviceWorkload.from_workload(w)
+    y = S.forward_stack(dw)
+    check(np_(y), oracle_stack(w), dtype, "Y edge lengths")
+
+
+def test_empty_batch_is_noop():
+    w = W.custom([0, 0], d=64, H=2, dtype="bf16")
+    dw = S.DeviceWorkload.from_workload(w)
+    y = S.forward_stack(dw)
+    assert y.shape == (0, 64)
+
+
+def test_large_time_gaps_saturate_bucket():
+    """Gaps of years (> 2^30 s) land in the last time bucket."""
+    lengths = [5]
+    ts = np.array([0, 1, 2 ** 31, 2 ** 31 + 5, 2 ** 40], np.int64)
+    w = W.custom(lengths, d=64, H=2, dtype="f32", timestamps=ts)
+    dw = S.DeviceWorkload.from_workload(w)
+    y = S.forward_stack(dw)
+    check(np_(y), oracle_stack(w), "f32", "Y large gaps")
+
+
+# ----------------------------------------------------------------------------
+# Validation flags and accounting
+# ----------------------------------------------------------------------------
+
+def test_validate_inputs_flags():
+    offs = torch.tensor([0, 3, 5, 9], dtype=torch.int64, device=DEV)
+    ts = torch.arange(9, dtype=torch.int64, device=DEV)
+    nt = torch.tensor([0, 2, 4], dtype=torch.int32, device=DEV)
+    assert H.validate_inputs(offs, ts, nt, 8192) == 0
+    bad = torch.tensor([1, 3, 2, 9], dtype=torch.int64, device=DEV)
+    f = H.validate_inputs(bad, ts, nt, 8192)
+    assert f & H.FLAG_OFFSETS_START and f & H.FLAG_OFFSETS_ORDER
+    assert H.validate_inputs(offs, ts, nt, 3) & H.FLAG_SEQ_TOO_LONG
+    assert H.validate_inputs(offs, ts, torch.tensor([0, 3, 4], dtype=torch.int32, device=DEV),
+                             8192) & H.FLAG_TARGETS_RANGE
+    ts2 = ts.clone()
+    ts2[6] = -5
+    assert H.validate_inputs(offs, ts2, nt, 8192) & H.FLAG_TIME_ORDER
+    short = torch.tensor([0, 3, 5, 8], dtype=torch.int64, device=DEV)
+    assert H.validate_inputs(short, ts, nt, 8192) & H.FLAG_OFFSETS_END
+
+
+def test_profiler_and_launch_count():
+    w = W.custom([100, 50], d=128, H=2, dtype="bf16")
+    dw = S.DeviceWorkload.from_workload(w)
+    H.profiler_reset()
+    H.profiler_enable(True)
+    S.forward_stack(dw)
+    torch.cuda.synchronize()
+    H.profiler_enable(False)
+    n, ms = H.profiler_collect(H.K_ATTN_FWD)
+    assert n == 1 and ms > 0
+    assert H.launch_count() >= 4

@@ -510,3 +510,39 @@ def test_pins_catch_planted_mistakes(monkeypatch, mutant):
     orig = getattr(R, attr)
     monkeypatch.setattr(R, attr, make(orig))
     assert _pin_suite() > 0, f"no pin caught mutant {mutant}"
+
+
+# ----------------------------------------------------------------------------
+# Single-step oracle functions compose back into the pinned layer
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("targets", [None, [3, 0, 6]])
+def test_step_functions_compose_to_layer(targets):
+    w = W.custom([9, 4, 6], d=16, H=2, dtype="f32", N=6.0, num_targets=targets, with_bias=True,
+                 with_affine=True, backward=True, mean_gap=250.0)
+    p = lp(w.params[0]).as_f64()
+    cfg = lcfg(w)
+    nt = w.num_targets
+    y, cache = R.layer_forward(w.x, w.seq_offsets, w.timestamps, nt, p, cfg, keep=True)
+    dx, gr = R.layer_backward(w.dy, w.seq_offsets, cache, p, cfg)
+    x = w.x.astype(np.float64)
+    d = 16
+    pre = x @ p.W1 + p.b1
+    g = R.silu(pre)
+    o = R.attention_forward(g, w.seq_offsets, w.timestamps, nt, p.rab_pos, p.rab_time, cfg)
+    z, mu, rstd = R.ln_gate_forward(o, g[:, :d], p.gamma, p.beta, cfg.ln_eps)
+    y2 = z @ p.W2 + p.b2 + x
+    np.testing.assert_allclose(y2, y, rtol=0, atol=1e-13)
+    dy = w.dy.astype(np.float64)
+    dz = dy @ p.W2.T
+    do, du, dgam, dbet = R.ln_gate_backward(dz, o, g[:, :d], p.gamma, p.beta, cfg.ln_eps)
+    dg, drp, drt = R.attention_backward(g, do, w.seq_offsets, w.timestamps, nt, p.rab_pos,
+                                        p.rab_time, cfg)
+    dg[:, :d] = du
+    dpre = dg * R.silu_grad(pre)
+    np.testing.assert_allclose(dpre @ p.W1.T + dy, dx, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(x.T @ dpre, gr.dW1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dgam, gr.dgamma, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dbet, gr.dbeta, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(drp, gr.drab_pos, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(drt, gr.drab_time, rtol=0, atol=1e-12)

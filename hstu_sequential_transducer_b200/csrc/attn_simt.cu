@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(256) attn_bwd_self_kernel(AttnBwdArgs A) {
   const float rp0 = a.rab_pos ? a.rab_pos[h * a.P] : 0.f;
   const float rt0 = a.rab_time ? a.rab_time[h * a.Bt] : 0.f;
   float dsum = 0.f;
-  for (int i = hlen + warp; i < n; i += nw) {
+  for (int i = max(hlen, 0) + warp; i < n; i += nw) {
     const int64_t t = s0 + i;
     float qv[DH / 32], kv[DH / 32], vv[DH / 32], dov[DH / 32];
     float sq = 0.f, sa = 0.f;

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) attn_fwd_simt_kernel(AttnArgs a) {
     qbase = nkv;
   } else {
     const int m = a.num_targets ? a.num_targets[b] : 0;
-    hlen = nq - m;
+    hlen = min(max(nq - m, 0), nq);  // clamped: malformed counts never index out of range
     qbase = 0;
   }
   const int rows = min(BQ, nq - r0);
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(256) attn_bwd_simt_kernel(AttnBwdArgs A) {
   const int64_t s0 = a.q_offsets[b];
   const int n = (int)(a.q_offsets[b + 1] - s0);
   const int m = a.num_targets ? a.num_targets[b] : 0;
-  const int hlen = n - m;
+  const int hlen = min(max(n - m, 0), n);
   if (k0 >= hlen) return;
   const int kn = min(BK, hlen - k0);
 
@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(256) attn_bwd_self_kernel(AttnBwdArgs A) {
   const int64_t s0 = a.q_offsets[b];
   const int n = (int)(a.q_offsets[b + 1] - s0);
   const int m = a.num_targets ? a.num_targets[b] : 0;
-  const int hlen = n - m;
+  const int hlen = min(max(n - m, 0), n);
   const int lane = threadIdx.x % 32;
   const int warp = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int nw = gridDim.x * (blockDim.x / 32);
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(256) attn_bwd_self_kernel(AttnBwdArgs A) {
   const float rp0 = a.rab_pos ? a.rab_pos[h * a.P] : 0.f;
   const float rt0 = a.rab_time ? a.rab_time[h * a.Bt] : 0.f;
   float dsum = 0.f;
-  for (int i = max(hlen, 0) + warp; i < n; i += nw) {
+  for (int i = hlen + warp; i < n; i += nw) {
     const int64_t t = s0 + i;
     float qv[DH / 32], kv[DH / 32], vv[DH / 32], dov[DH / 32];
     float sq = 0.f, sa = 0.f;

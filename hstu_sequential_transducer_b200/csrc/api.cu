@@ -47,6 +47,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 hstu_status check_cfg(const hstu_config* c) {
   if (!c) return HSTU_ERR_INVALID;
   if (c->dtype != HSTU_F32 && c->dtype != HSTU_BF16) return HSTU_ERR_INVALID;
+  if (c->io_dtype != HSTU_F32 && c->io_dtype != HSTU_BF16) return HSTU_ERR_INVALID;
+  if (c->io_dtype != c->dtype && !(c->dtype == HSTU_BF16 && c->io_dtype == HSTU_F32))
+    return HSTU_ERR_UNSUPPORTED;
   if (c->d_model <= 0 || c->num_heads <= 0 || c->head_dim <= 0) return HSTU_ERR_INVALID;
   if (c->num_heads * c->head_dim != c->d_model) return HSTU_ERR_INVALID;
   if (!(c->norm_N > 0.f) || !std::isfinite(c->norm_N)) return HSTU_ERR_INVALID;
@@ -93,8 +96,9 @@ void saved_offsets(const hstu_config* c, int64_t T, size_t off[HSTU_SAVED_COUNT 
   const size_t es = (size_t)dtype_size(c->dtype);
   const size_t d = (size_t)c->d_model;
   const size_t t = (size_t)T;
-  const size_t sizes[HSTU_SAVED_COUNT] = {t * 4 * d * es, t * 4 * d * es, t * d * es,
-                                          t * d * es,     t * 4,          t * 4};
+  const size_t xlow = c->io_dtype != c->dtype ? t * d * es : 0;
+  const size_t sizes[HSTU_SAVED_COUNT] = {t * 4 * d * es, t * 4 * d * es, t * d * 4,
+                                          t * d * es,     t * 4,          t * 4, xlow};
   size_t o = 0;
   for (int i = 0; i < HSTU_SAVED_COUNT; ++i) {
     off[i] = o;
@@ -104,7 +108,7 @@ void saved_offsets(const hstu_config* c, int64_t T, size_t off[HSTU_SAVED_COUNT 
 }
 
 struct FwdWs {
-  size_t g, o, z, attn, total;
+  size_t g, o, z, xlow, attn, total;
 };
 FwdWs fwd_ws(const hstu_config* c, int B, int64_t T) {
   const size_t es = (size_t)dtype_size(c->dtype), d = (size_t)c->d_model;
@@ -112,14 +116,15 @@ FwdWs fwd_ws(const hstu_config* c, int B, int64_t T) {
   FwdWs w;
   w.g = 0;
   w.o = align_up(w.g + t * 4 * d * es, 256);
-  w.z = align_up(w.o + t * d * es, 256);
-  w.attn = align_up(w.z + t * d * es, 256);
+  w.z = align_up(w.o + t * d * 4, 256);
+  w.xlow = align_up(w.z + t * d * es, 256);
+  w.attn = align_up(w.xlow + (c->io_dtype != c->dtype ? t * d * es : 0), 256);
   w.total = align_up(w.attn + attention_fwd_ws(B, T, c->num_heads, c->max_seq_len), 256);
   return w;
 }
 
 struct BwdWs {
-  size_t dz, dO, dpre, dq, attn, total;
+  size_t dz, dO, dpre, dq, dylow, attn, total;
 };
 BwdWs bwd_ws(const hstu_config* c, int B, int64_t T) {
   const size_t es = (size_t)dtype_size(c->dtype), d = (size_t)c->d_model;
@@ -129,7 +134,8 @@ BwdWs bwd_ws(const hstu_config* c, int B, int64_t T) {
   w.dO = align_up(w.dz + t * d * es, 256);
   w.dpre = align_up(w.dO + t * d * es, 256);
   w.dq = align_up(w.dpre + t * 4 * d * es, 256);
-  w.attn = align_up(w.dq + t * d * 4, 256);
+  w.dylow = align_up(w.dq + t * d * 4, 256);
+  w.attn = align_up(w.dylow + (c->io_dtype != c->dtype ? t * d * es : 0), 256);
   w.total = align_up(w.attn + attention_bwd_ws(B, T, c->num_heads, c->d_model, c->max_seq_len), 256);
   return w;
 }
@@ -197,7 +203,8 @@ hstu_status do_ln_fwd(const hstu_config* c, const void* gamma, const void* beta,
                       const void* g, int64_t T, void* z, float* mean, float* rstd,
                       cudaStream_t s) {
   prof_begin(HSTU_K_LN_FWD, s);
-  cudaError_t e = ln_gate_fwd(c->dtype, c->d_model, c->ln_eps, gamma, beta, o, g,
+  cudaError_t e = ln_gate_fwd(c->dtype, c->d_model, c->ln_eps, gamma, beta,
+                              static_cast<const float*>(o), g,
                               4 * (int64_t)c->d_model, T, z, mean, rstd, s);
   prof_end(HSTU_K_LN_FWD, s);
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
@@ -211,6 +218,7 @@ hstu_status do_proj_out(const hstu_config* c, const void* W2, const void* b2, co
   a.B = W2; a.ldb = d; a.b_kmajor = false;
   a.M = T; a.N = d; a.K = d;
   a.epi = x ? EPI_RESID : EPI_STORE; a.C = y; a.ldc = d; a.bias = b2; a.R = x; a.ldr = d;
+  a.io_f32 = c->io_dtype == HSTU_F32;
   prof_begin(HSTU_K_PROJ_OUT, s);
   cudaError_t e = gemm(c->dtype, a, s);
   prof_end(HSTU_K_PROJ_OUT, s);
@@ -245,7 +253,8 @@ hstu_status do_ln_bwd(const hstu_config* c, const void* gamma, const void* beta,
                       const float* rstd, int64_t T, void* dO, void* dpre, float* dgamma,
                       float* dbeta, cudaStream_t s) {
   prof_begin(HSTU_K_LN_BWD, s);
-  cudaError_t e = ln_gate_bwd(c->dtype, c->d_model, gamma, beta, dz, o, g, pre,
+  cudaError_t e = ln_gate_bwd(c->dtype, c->d_model, gamma, beta, dz,
+                              static_cast<const float*>(o), g, pre,
                               4 * (int64_t)c->d_model, mean, rstd, T, dO, dpre, dgamma, dbeta, s);
   prof_end(HSTU_K_LN_BWD, s);
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
@@ -292,6 +301,7 @@ hstu_status do_proj_in_bwd(const hstu_config* c, const void* W1, const void* x, 
   a.B = W1; a.ldb = 4 * d; a.b_kmajor = true;
   a.M = T; a.N = d; a.K = 4 * d;
   a.epi = dy ? EPI_RESID : EPI_STORE; a.C = dx; a.ldc = d; a.R = dy; a.ldr = d;
+  a.io_f32 = c->io_dtype == HSTU_F32;
   cudaError_t e = cudaSuccess;
   // dW1 first: dx may alias dy but never x or dpre
   if (dW1) {
@@ -305,6 +315,20 @@ hstu_status do_proj_in_bwd(const hstu_config* c, const void* W1, const void* x, 
   if (e == cudaSuccess && db1) e = colsum_accumulate(c->dtype, dpre, T, 4 * d, 4 * d, db1, s);
   if (e == cudaSuccess) e = gemm(c->dtype, a, s);
   prof_end(HSTU_K_PROJ_IN_BWD, s);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// x (io dtype) -> operand dtype copy when the two differ; returns the operand pointer.
+hstu_status to_operand(const hstu_config* c, const void* x, int64_t rows, void* low,
+                       const void** out, cudaStream_t s) {
+  if (c->io_dtype == c->dtype) {
+    *out = x;
+    return HSTU_OK;
+  }
+  prof_begin(HSTU_K_MISC, s);
+  cudaError_t e = convert_f32_to_bf16(static_cast<const float*>(x), low, rows * c->d_model, s);
+  prof_end(HSTU_K_MISC, s);
+  *out = low;
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
@@ -657,7 +681,7 @@ hstu_status hstu_fwd(const hstu_config* cfg, const hstu_weights* w, const void* 
   if (T == 0 || B == 0) return HSTU_OK;
   HSTU_TRY(need(workspace, 1));
   const int d = cfg->d_model, es = dtype_size(cfg->dtype);
-  void *pre = nullptr, *g, *o, *z;
+  void *pre = nullptr, *g, *o, *z, *xlow = at(workspace, L.xlow);
   float *mean = nullptr, *rstd = nullptr;
   if (saved) {
     size_t off[HSTU_SAVED_COUNT + 1];
@@ -668,12 +692,15 @@ hstu_status hstu_fwd(const hstu_config* cfg, const hstu_weights* w, const void* 
     z = at(saved, off[HSTU_SAVED_Z]);
     mean = reinterpret_cast<float*>(at(saved, off[HSTU_SAVED_MEAN]));
     rstd = reinterpret_cast<float*>(at(saved, off[HSTU_SAVED_RSTD]));
+    xlow = at(saved, off[HSTU_SAVED_XLOW]);
   } else {
     g = at(workspace, L.g);
     o = at(workspace, L.o);
     z = at(workspace, L.z);
   }
-  HSTU_TRY(do_proj_in(cfg, w->W1, w->b1, x, T, pre, g, stream));
+  const void* xop = nullptr;
+  HSTU_TRY(to_operand(cfg, x, T, xlow, &xop, stream));
+  HSTU_TRY(do_proj_in(cfg, w->W1, w->b1, xop, T, pre, g, stream));
   AttnArgs a = full_attn_args(cfg, w->rab_pos, w->rab_time, g, seq_offsets, B, timestamps,
                               num_targets, o);
   HSTU_TRY(do_attention_fwd(cfg, a, at(workspace, L.attn), ws_bytes - L.attn, stream,
@@ -714,7 +741,9 @@ hstu_status hstu_fwd_cached(const hstu_config* cfg, const hstu_weights* w, const
   void* g = at(workspace, L.g);
   void* o = at(workspace, L.o);
   void* z = at(workspace, L.z);
-  HSTU_TRY(do_proj_in(cfg, w->W1, w->b1, cand_x, Tc, nullptr, g, stream));
+  const void* xop = nullptr;
+  HSTU_TRY(to_operand(cfg, cand_x, Tc, at(workspace, L.xlow), &xop, stream));
+  HSTU_TRY(do_proj_in(cfg, w->W1, w->b1, xop, Tc, nullptr, g, stream));
   AttnArgs a = full_attn_args(cfg, w->rab_pos, w->rab_time, g, cand_offsets, B, cand_timestamps,
                               nullptr, o);
   a.cached = 1;
@@ -764,13 +793,16 @@ hstu_status hstu_bwd(const hstu_config* cfg, const hstu_weights* w, const void* 
   void* dO = at(workspace, L.dO);
   void* dpre = at(workspace, L.dpre);
   float* dq = reinterpret_cast<float*>(at(workspace, L.dq));
-  HSTU_TRY(do_proj_out_bwd(cfg, w->W2, z, dy, T, dz, gr.dW2, gr.db2, stream));
+  const void* xop = cfg->io_dtype == cfg->dtype ? x : at(svd, off[HSTU_SAVED_XLOW]);
+  const void* dyop = nullptr;
+  HSTU_TRY(to_operand(cfg, dy, T, at(workspace, L.dylow), &dyop, stream));
+  HSTU_TRY(do_proj_out_bwd(cfg, w->W2, z, dyop, T, dz, gr.dW2, gr.db2, stream));
   HSTU_TRY(do_ln_bwd(cfg, w->ln_gamma, w->ln_beta, dz, o, g, pre, mean, rstd, T, dO, dpre,
                      gr.dgamma, gr.dbeta, stream));
   HSTU_TRY(do_attention_bwd(cfg, w->rab_pos, w->rab_time, g, pre, dO, seq_offsets, B, T,
                             timestamps, num_targets, dpre, gr.drab_pos, gr.drab_time, dq,
                             at(workspace, L.attn), ws_bytes - L.attn, stream));
-  HSTU_TRY(do_proj_in_bwd(cfg, w->W1, x, dpre, dy, T, dx, gr.dW1, gr.db1, stream));
+  HSTU_TRY(do_proj_in_bwd(cfg, w->W1, xop, dpre, dy, T, dx, gr.dW1, gr.db1, stream));
   return HSTU_OK;
 }
 

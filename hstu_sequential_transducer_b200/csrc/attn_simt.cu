@@ -164,14 +164,14 @@ __global__ void __launch_bounds__(256) attn_fwd_simt_kernel(AttnArgs a) {
     }
   }
 
-  T* O = static_cast<T*>(a.o);
+  float* O = static_cast<float*>(a.o);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     if (!rvalid[i]) continue;
     const int r = ty * 4 + i;
 #pragma unroll
     for (int j = 0; j < DH / 16; ++j)
-      O[(qs + r0 + r) * a.o_stride + h * DH + tx + 16 * j] = from_f<T>(acc[i][j] * a.inv_N);
+      O[(qs + r0 + r) * a.o_stride + h * DH + tx + 16 * j] = acc[i][j] * a.inv_N;
   }
 }
 

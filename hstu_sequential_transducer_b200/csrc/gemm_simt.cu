@@ -11,7 +11,7 @@ namespace {
 
 constexpr int TM = 64, TN = 64, TK = 16;
 
-template <typename T, bool AK, bool BK, int EPI>
+template <typename T, bool AK, bool BK, int EPI, typename TIO>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g, int64_t k_per_split) {
   __shared__ float As[TK][TM + 4];
   __shared__ float Bs[TK][TN + 4];
@@ -76,8 +76,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs g, int64_t k_pe
         if (g.C) static_cast<T*>(g.C)[m * g.ldc + n] = from_f<T>(v);
         static_cast<T*>(g.C2)[m * g.ldc + n] = from_f<T>(silu_acc(v));
       } else {
-        if (EPI == EPI_RESID) v += to_f(static_cast<const T*>(g.R)[m * g.ldr + n]);
-        static_cast<T*>(g.C)[m * g.ldc + n] = from_f<T>(v);
+        if (EPI == EPI_RESID) v += to_f(static_cast<const TIO*>(g.R)[m * g.ldr + n]);
+        static_cast<TIO*>(g.C)[m * g.ldc + n] = from_f<TIO>(v);
       }
     }
   }
@@ -100,10 +100,16 @@ cudaError_t launch_epi(const GemmArgs& g, cudaStream_t s) {
   }
   if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
   switch (g.epi) {
-    case EPI_STORE: gemm_simt_kernel<T, AK, BK, EPI_STORE><<<grid, 256, 0, s>>>(g, kps); break;
-    case EPI_SILU_SPLIT: gemm_simt_kernel<T, AK, BK, EPI_SILU_SPLIT><<<grid, 256, 0, s>>>(g, kps); break;
-    case EPI_RESID: gemm_simt_kernel<T, AK, BK, EPI_RESID><<<grid, 256, 0, s>>>(g, kps); break;
-    case EPI_ATOMIC_F32: gemm_simt_kernel<T, AK, BK, EPI_ATOMIC_F32><<<grid, 256, 0, s>>>(g, kps); break;
+    case EPI_STORE:
+      if (g.io_f32) gemm_simt_kernel<T, AK, BK, EPI_STORE, float><<<grid, 256, 0, s>>>(g, kps);
+      else gemm_simt_kernel<T, AK, BK, EPI_STORE, T><<<grid, 256, 0, s>>>(g, kps);
+      break;
+    case EPI_SILU_SPLIT: gemm_simt_kernel<T, AK, BK, EPI_SILU_SPLIT, T><<<grid, 256, 0, s>>>(g, kps); break;
+    case EPI_RESID:
+      if (g.io_f32) gemm_simt_kernel<T, AK, BK, EPI_RESID, float><<<grid, 256, 0, s>>>(g, kps);
+      else gemm_simt_kernel<T, AK, BK, EPI_RESID, T><<<grid, 256, 0, s>>>(g, kps);
+      break;
+    case EPI_ATOMIC_F32: gemm_simt_kernel<T, AK, BK, EPI_ATOMIC_F32, T><<<grid, 256, 0, s>>>(g, kps); break;
     default: return cudaErrorInvalidValue;
   }
   count_launch();

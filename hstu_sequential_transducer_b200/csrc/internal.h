@@ -35,6 +35,7 @@ struct GemmArgs {
   const void* bias = nullptr;  // [N] dtype
   const void* R = nullptr;     // residual, row-major ldr (EPI_RESID)
   int64_t ldr = 0;
+  bool io_f32 = false;         // C (EPI_STORE / EPI_RESID) and R are fp32 whatever the operands
   float* Cf = nullptr;      // fp32 accumulation target, row-major ldc (EPI_ATOMIC_F32)
 };
 
@@ -54,7 +55,7 @@ struct AttnArgs {
   const void* k = nullptr;
   const void* v = nullptr;
   int64_t kv_stride = 0;
-  void* o = nullptr;             // [T_q][d]
+  void* o = nullptr;             // [T_q][d] fp32
   int64_t o_stride = 0;
   const int64_t* q_offsets = nullptr;
   const int64_t* kv_offsets = nullptr;
@@ -91,10 +92,10 @@ size_t attention_bwd_ws(int B, int64_t T, int H, int d, int max_len);
 // LayerNorm (.) U epilogue
 // ---------------------------------------------------------------------------
 cudaError_t ln_gate_fwd(int dtype, int d, float eps, const void* gamma, const void* beta,
-                        const void* o, const void* g, int64_t g_stride, int64_t T, void* z,
+                        const float* o, const void* g, int64_t g_stride, int64_t T, void* z,
                         float* mean, float* rstd, cudaStream_t s);
 cudaError_t ln_gate_bwd(int dtype, int d, const void* gamma, const void* beta, const void* dz,
-                        const void* o, const void* g, const void* pre, int64_t g_stride,
+                        const float* o, const void* g, const void* pre, int64_t g_stride,
                         const float* mean, const float* rstd, int64_t T, void* dout, void* dpre,
                         float* dgamma, float* dbeta, cudaStream_t s);
 
@@ -107,6 +108,7 @@ cudaError_t dq_finalize(int dtype, const float* dq_acc, const void* pre_q, int64
                         void* dpre_q, int64_t T, int d, cudaStream_t s);
 cudaError_t copy_columns(int dtype, const void* src, int64_t src_stride, void* dst,
                          int64_t dst_stride, int64_t rows, int64_t cols, cudaStream_t s);
+cudaError_t convert_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t s);
 cudaError_t validate_inputs(const int64_t* offs, int B, int64_t T, const int64_t* ts,
                             const int32_t* nt, int max_len, uint32_t* flags, cudaStream_t s);
 

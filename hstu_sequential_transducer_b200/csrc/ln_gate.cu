@@ -49,11 +49,20 @@ template <> struct Vec<float> {
   }
 };
 
+template <int N>
+__device__ __forceinline__ void load_f32(const float* p, float* f) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4) {
+    const float4 u = *reinterpret_cast<const float4*>(p + i);
+    f[i] = u.x; f[i + 1] = u.y; f[i + 2] = u.z; f[i + 3] = u.w;
+  }
+}
+
 // CH = vector chunks per lane (d <= 32 * CH * VEC)
 template <typename T, int CH>
 __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, const T* __restrict__ gamma,
                                                           const T* __restrict__ beta,
-                                                          const T* __restrict__ o,
+                                                          const float* __restrict__ o,
                                                           const T* __restrict__ g, int64_t g_stride,
                                                           int64_t rows, T* __restrict__ z,
                                                           float* __restrict__ mean_out,
@@ -82,7 +91,7 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
     for (int c = 0; c < CH; ++c) {
       const int ch = lane + 32 * c;
       if (ch < nchunk) {
-        Vec<T>::load(o + r * d + ch * VN, x[c]);
+        load_f32<VN>(o + r * d + ch * VN, x[c]);
 #pragma unroll
         for (int k = 0; k < VN; ++k) s += x[c][k];
       } else {
@@ -121,7 +130,7 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
 template <typename T, int CH>
 __global__ void __launch_bounds__(256) ln_gate_bwd_kernel(
     int d, const T* __restrict__ gamma, const T* __restrict__ beta, const T* __restrict__ dz,
-    const T* __restrict__ o, const T* __restrict__ g, const T* __restrict__ pre, int64_t g_stride,
+    const float* __restrict__ o, const T* __restrict__ g, const T* __restrict__ pre, int64_t g_stride,
     const float* __restrict__ mean, const float* __restrict__ rstd, int64_t rows,
     T* __restrict__ dout, T* __restrict__ dpre, float* __restrict__ dgamma,
     float* __restrict__ dbeta) {
@@ -154,7 +163,7 @@ __global__ void __launch_bounds__(256) ln_gate_bwd_kernel(
       const int ch = lane + 32 * c;
       if (ch < nchunk) {
         float x[VN], gz[VN], u[VN], pu[VN], du[VN];
-        Vec<T>::load(o + r * d + ch * VN, x);
+        load_f32<VN>(o + r * d + ch * VN, x);
         Vec<T>::load(dz + r * d + ch * VN, gz);
         Vec<T>::load(g + r * g_stride + ch * VN, u);
         Vec<T>::load(pre + r * g_stride + ch * VN, pu);
@@ -220,7 +229,7 @@ int num_sms() {
 }
 
 template <typename T, int CH>
-cudaError_t fwd_ch(int d, float eps, const void* gamma, const void* beta, const void* o,
+cudaError_t fwd_ch(int d, float eps, const void* gamma, const void* beta, const float* o,
                    const void* g, int64_t gs, int64_t T_, void* z, float* mean, float* rstd,
                    cudaStream_t s) {
   int64_t blocks = (T_ + 7) / 8;
@@ -228,13 +237,13 @@ cudaError_t fwd_ch(int d, float eps, const void* gamma, const void* beta, const 
   if (blocks > cap) blocks = cap;
   if (blocks == 0) return cudaSuccess;
   ln_gate_fwd_kernel<T, CH><<<(unsigned)blocks, 256, 0, s>>>(
-      d, eps, (const T*)gamma, (const T*)beta, (const T*)o, (const T*)g, gs, T_, (T*)z, mean, rstd);
+      d, eps, (const T*)gamma, (const T*)beta, o, (const T*)g, gs, T_, (T*)z, mean, rstd);
   count_launch();
   return cudaGetLastError();
 }
 
 template <typename T, int CH>
-cudaError_t bwd_ch(int d, const void* gamma, const void* beta, const void* dz, const void* o,
+cudaError_t bwd_ch(int d, const void* gamma, const void* beta, const void* dz, const float* o,
                    const void* g, const void* pre, int64_t gs, const float* mean, const float* rstd,
                    int64_t T_, void* dout, void* dpre, float* dgamma, float* dbeta, cudaStream_t s) {
   int64_t blocks = (T_ + 7) / 8;
@@ -242,7 +251,7 @@ cudaError_t bwd_ch(int d, const void* gamma, const void* beta, const void* dz, c
   if (blocks > cap) blocks = cap;
   if (blocks == 0) return cudaSuccess;
   ln_gate_bwd_kernel<T, CH><<<(unsigned)blocks, 256, 2 * d * sizeof(float), s>>>(
-      d, (const T*)gamma, (const T*)beta, (const T*)dz, (const T*)o, (const T*)g, (const T*)pre, gs,
+      d, (const T*)gamma, (const T*)beta, (const T*)dz, o, (const T*)g, (const T*)pre, gs,
       mean, rstd, T_, (T*)dout, (T*)dpre, dgamma, dbeta);
   count_launch();
   return cudaGetLastError();
@@ -251,7 +260,7 @@ cudaError_t bwd_ch(int d, const void* gamma, const void* beta, const void* dz, c
 }  // namespace
 
 cudaError_t ln_gate_fwd(int dtype, int d, float eps, const void* gamma, const void* beta,
-                        const void* o, const void* g, int64_t gs, int64_t T_, void* z, float* mean,
+                        const float* o, const void* g, int64_t gs, int64_t T_, void* z, float* mean,
                         float* rstd, cudaStream_t s) {
   const int vn = dtype == HSTU_BF16 ? 8 : 4;
   const int ch = (d / vn + 31) / 32;
@@ -270,7 +279,7 @@ cudaError_t ln_gate_fwd(int dtype, int d, float eps, const void* gamma, const vo
 }
 
 cudaError_t ln_gate_bwd(int dtype, int d, const void* gamma, const void* beta, const void* dz,
-                        const void* o, const void* g, const void* pre, int64_t gs,
+                        const float* o, const void* g, const void* pre, int64_t gs,
                         const float* mean, const float* rstd, int64_t T_, void* dout, void* dpre,
                         float* dgamma, float* dbeta, cudaStream_t s) {
   const int vn = dtype == HSTU_BF16 ? 8 : 4;

@@ -51,6 +51,25 @@ __global__ void copy_columns_kernel(const T* __restrict__ src, int64_t ss, T* __
   }
 }
 
+__global__ void convert_kernel(const float* __restrict__ src, bf16* __restrict__ dst, int64_t n) {
+  const int64_t n8 = n / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(src)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(src)[2 * i + 1];
+    uint4 o;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+    h[0] = __floats2bfloat162_rn(a.x, a.y);
+    h[1] = __floats2bfloat162_rn(a.z, a.w);
+    h[2] = __floats2bfloat162_rn(b.x, b.y);
+    h[3] = __floats2bfloat162_rn(b.z, b.w);
+    reinterpret_cast<uint4*>(dst)[i] = o;
+  }
+  for (int64_t i = n8 * 8 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
 __global__ void validate_seq_kernel(const int64_t* __restrict__ offs, int B, int64_t T,
                                     const int32_t* __restrict__ nt, int max_len,
                                     uint32_t* __restrict__ flags) {
@@ -127,6 +146,13 @@ cudaError_t copy_columns(int dtype, const void* src, int64_t ss, void* dst, int6
     copy_columns_kernel<bf16><<<g, 256, 0, s>>>((const bf16*)src, ss, (bf16*)dst, ds, rows, cols);
   else
     copy_columns_kernel<float><<<g, 256, 0, s>>>((const float*)src, ss, (float*)dst, ds, rows, cols);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t convert_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  convert_kernel<<<grid_for(n / 8 + 1, 256), 256, 0, s>>>(src, (bf16*)dst, n);
   count_launch();
   return cudaGetLastError();
 }

@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libhstu.so")
 
 HSTU_F32, HSTU_BF16 = 0, 1
-SAVED_PRE, SAVED_G, SAVED_O, SAVED_Z, SAVED_MEAN, SAVED_RSTD, SAVED_COUNT = range(7)
+SAVED_PRE, SAVED_G, SAVED_O, SAVED_Z, SAVED_MEAN, SAVED_RSTD, SAVED_XLOW, SAVED_COUNT = range(8)
 K_PROJ_IN, K_ATTN_FWD, K_LN_FWD, K_PROJ_OUT, K_PROJ_OUT_BWD, K_LN_BWD, K_ATTN_BWD, \
     K_PROJ_IN_BWD, K_ATTN_CACHED, K_MISC, K_COUNT = range(11)
 KERNEL_NAMES = ["proj_in", "attn_fwd", "ln_fwd", "proj_out", "proj_out_bwd", "ln_bwd",
@@ -33,7 +33,7 @@ class Config(Structure):
     _fields_ = [("d_model", c_int32), ("num_heads", c_int32), ("head_dim", c_int32),
                 ("num_pos_buckets", c_int32), ("num_time_buckets", c_int32),
                 ("max_seq_len", c_int32), ("norm_N", c_float), ("ln_eps", c_float),
-                ("dtype", c_int32)]
+                ("dtype", c_int32), ("io_dtype", c_int32)]
 
 
 class Weights(Structure):
@@ -133,9 +133,12 @@ def torch_dtype(dtype: int):
 
 def make_config(d_model: int, num_heads: int, norm_N: float, dtype: int = HSTU_BF16,
                 num_pos_buckets: int = 32, num_time_buckets: int = 32, max_seq_len: int = 8192,
-                ln_eps: float = 1e-5) -> Config:
+                ln_eps: float = 1e-5, io_dtype: Optional[int] = None) -> Config:
+    """io_dtype (x, y, dy, dx) defaults to fp32: a bf16 layer then keeps its
+    residual stream in fp32 and only the contraction operands are bf16."""
+    io = HSTU_F32 if io_dtype is None else io_dtype
     return Config(d_model, num_heads, d_model // num_heads, num_pos_buckets, num_time_buckets,
-                  max_seq_len, float(norm_N), float(ln_eps), dtype)
+                  max_seq_len, float(norm_N), float(ln_eps), dtype, io)
 
 
 @dataclass
@@ -204,12 +207,15 @@ def saved_views(cfg: Config, saved: torch.Tensor, T: int):
     def view(i, n, dtype, shape):
         nbytes = n * (4 if dtype == torch.float32 else es)
         return saved[off[i]:off[i] + nbytes].view(dtype).view(*shape)
-    return {"pre": view(SAVED_PRE, T * 4 * d, dt, (T, 4 * d)),
+    out = {"pre": view(SAVED_PRE, T * 4 * d, dt, (T, 4 * d)),
             "g": view(SAVED_G, T * 4 * d, dt, (T, 4 * d)),
-            "o": view(SAVED_O, T * d, dt, (T, d)),
+            "o": view(SAVED_O, T * d, torch.float32, (T, d)),
             "z": view(SAVED_Z, T * d, dt, (T, d)),
             "mean": view(SAVED_MEAN, T, torch.float32, (T,)),
             "rstd": view(SAVED_RSTD, T, torch.float32, (T,))}
+    if cfg.io_dtype != cfg.dtype:
+        out["xlow"] = view(SAVED_XLOW, T * d, dt, (T, d))
+    return out
 
 
 _ws_cache = {}

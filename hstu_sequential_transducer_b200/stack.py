@@ -33,11 +33,15 @@ class DeviceWorkload:
     w: Workload
 
     @staticmethod
-    def from_workload(w: Workload, device="cuda", with_targets=True) -> "DeviceWorkload":
+    def from_workload(w: Workload, device="cuda", with_targets=True,
+                      io_dtype: int = H.HSTU_F32) -> "DeviceWorkload":
+        """io_dtype: dtype of the residual stream (x, y, dy, dx)."""
         dtype_id = H.HSTU_BF16 if w.dtype == "bf16" else H.HSTU_F32
         dt = H.torch_dtype(dtype_id)
+        io_dt = H.torch_dtype(io_dtype)
         cfg = H.make_config(w.d_model, w.num_heads, w.norm_N, dtype_id, w.num_pos_buckets,
-                            w.num_time_buckets, max(int(w.lengths.max(initial=1)), 1), w.ln_eps)
+                            w.num_time_buckets, max(int(w.lengths.max(initial=1)), 1), w.ln_eps,
+                            io_dtype=io_dtype)
         layers = []
         for p in w.params:
             layers.append(H.LayerWeights(
@@ -48,9 +52,9 @@ class DeviceWorkload:
                 ln_gamma=_t(p.gamma, dt, device), ln_beta=_t(p.beta, dt, device)))
         nt = _t(w.num_targets, torch.int32, device) if (with_targets and w.num_targets is not None) \
             else None
-        return DeviceWorkload(cfg, _t(w.x, dt, device), _t(w.seq_offsets, torch.int64, device),
+        return DeviceWorkload(cfg, _t(w.x, io_dt, device), _t(w.seq_offsets, torch.int64, device),
                               _t(w.timestamps, torch.int64, device), nt, layers,
-                              _t(w.dy, dt, device), w)
+                              _t(w.dy, io_dt, device), w)
 
     @property
     def B(self):
@@ -144,7 +148,7 @@ def mfalcon_score(dw: DeviceWorkload, history: int, candidates: int, microbatch:
     caches = []
     y = x_hist
     for lw in dw.layers:
-        kv = torch.empty(y.shape[0], 2 * d, dtype=y.dtype, device=dev)
+        kv = torch.empty(y.shape[0], 2 * d, dtype=H.torch_dtype(dw.cfg.dtype), device=dev)
         y = H.fwd(dw.cfg, lw, y, hist_off, ts_hist, None, kv_out=kv, stream=stream)
         caches.append(kv)
     y_hist = y

@@ -41,7 +41,11 @@
  *     Launch failures return HSTU_ERR_CUDA.  Malformed *data* (offsets,
  *     timestamps, num_targets) is only detected by hstu_validate_inputs; the
  *     compute kernels assume validated data and never trap.
- *   - Activations are row-major [T][width] in cfg->dtype (fp32 or bf16).
+ *   - Internal activations (Pre, G, O, Z, dO, ...) are row-major [T][width]
+ *     in cfg->dtype (fp32 or bf16).  The layer boundary tensors x, y, dy, dx
+ *     (the residual stream) are in cfg->io_dtype, which may be fp32 while
+ *     cfg->dtype is bf16: the stream then keeps fp32 precision across a stack
+ *     of layers and only the operands of the contractions are bf16.
  *     Jagged sequences are concatenated: sequence b owns rows
  *     [seq_offsets[b], seq_offsets[b+1]); seq_offsets is int64 [B+1] with
  *     seq_offsets[0] = 0 and seq_offsets[B] = T.  timestamps is int64 [T]
@@ -89,7 +93,10 @@ typedef struct {
   int32_t max_seq_len;      /* upper bound on any sequence length (<= 65536)   */
   float norm_N;             /* the 1/N normaliser of equation (2)              */
   float ln_eps;             /* LayerNorm epsilon                               */
-  int32_t dtype;            /* hstu_dtype of activations and weights           */
+  int32_t dtype;            /* hstu_dtype of weights, internal activations and
+                               contraction operands                            */
+  int32_t io_dtype;         /* hstu_dtype of x, y, dy, dx; must equal dtype
+                               unless dtype is bf16 and io_dtype fp32         */
 } hstu_config;
 
 /* One layer's parameters (device pointers; see conventions for NULLs). */
@@ -117,12 +124,17 @@ typedef struct {
 } hstu_grads;
 
 /* Activations a training forward keeps for the backward (see
- * hstu_saved_layout): Pre = X W1 + b1 [T][4d], G = SiLU(Pre) [T][4d] (U|V|Q|K),
- * O [T][d], Z = LN(O) (.) U [T][d] in cfg->dtype, then mean [T] and rstd [T]
- * in fp32.  10*d activation elements plus 8 bytes per token. */
+ * hstu_saved_layout): Pre = X W1 + b1 [T][4d], G = SiLU(Pre) [T][4d] (U|V|Q|K)
+ * in cfg->dtype, O [T][d] in fp32, Z = LN(O) (.) U [T][d] in cfg->dtype, then
+ * mean [T] and rstd [T] in fp32, then (only when io_dtype differs from dtype)
+ * X rounded to cfg->dtype [T][d].
+ *
+ * O is always fp32: LayerNorm subtracts each row's mean, and the rows of O
+ * have a mean many times their spread (SiLU weights and values are mostly
+ * positive), so a bf16 O would lose the deviations LayerNorm keeps. */
 typedef enum {
   HSTU_SAVED_PRE = 0, HSTU_SAVED_G = 1, HSTU_SAVED_O = 2, HSTU_SAVED_Z = 3,
-  HSTU_SAVED_MEAN = 4, HSTU_SAVED_RSTD = 5, HSTU_SAVED_COUNT = 6
+  HSTU_SAVED_MEAN = 4, HSTU_SAVED_RSTD = 5, HSTU_SAVED_XLOW = 6, HSTU_SAVED_COUNT = 7
 } hstu_saved_part;
 
 /* ------------------------------------------------------------------------ */
@@ -145,14 +157,15 @@ hstu_status hstu_saved_layout(const hstu_config* cfg, int64_t T,
 /* ------------------------------------------------------------------------ */
 
 /* Equation (1): Pre = X W1 + b1 and G = SiLU(Pre), split as U|V|Q|K.
- * x [T][d]; pre_out [T][4d] may be NULL (inference); g_out [T][4d]. */
+ * x [T][d] in cfg->dtype (the contraction operand); pre_out [T][4d] may be
+ * NULL (inference); g_out [T][4d]. */
 hstu_status hstu_proj_in_fwd(const hstu_config* cfg, const hstu_weights* w,
                              const void* x, int64_t T, void* pre_out, void* g_out,
                              cudaStream_t stream);
 
 /* Equation (2) for every head, with rab^{p,t} bucketing, the causal or
  * M-FALCON mask, and ragged work partitioning (no padding is computed).
- * g [T][4d] holds U|V|Q|K of every token; o_out [T][d].
+ * g [T][4d] holds U|V|Q|K of every token; o_out [T][d] fp32.
  * workspace: at least hstu_attention_workspace_size(B, T) bytes. */
 hstu_status hstu_attention_fwd(const hstu_config* cfg, const float* rab_pos,
                                const float* rab_time, const void* g,
@@ -166,7 +179,7 @@ hstu_status hstu_attention_fwd(const hstu_config* cfg, const float* rab_pos,
  * to every cached history token of that user (hist_kv rows
  * [hist_offsets[b], hist_offsets[b+1]), layout [T_hist][2d] = V|K) and to
  * themselves, never to other candidates.  A candidate's position is the
- * user's history length.  o_out [Tc][d]. */
+ * user's history length.  o_out [Tc][d] fp32. */
 hstu_status hstu_attention_fwd_cached(const hstu_config* cfg, const float* rab_pos,
                                       const float* rab_time, const void* cand_g,
                                       const int64_t* cand_offsets, int32_t B, int64_t Tc,
@@ -179,24 +192,25 @@ hstu_status hstu_attention_fwd_cached(const hstu_config* cfg, const float* rab_p
 size_t hstu_attention_workspace_size(const hstu_config* cfg, int32_t B, int64_t T);
 
 /* Equation (3), first half: Z = (LayerNorm(O) * gamma + beta) (.) U.
- * o [T][d], g [T][4d] (U = columns [0, d)), z_out [T][d];
+ * o [T][d] fp32, g [T][4d] (U = columns [0, d)), z_out [T][d];
  * mean_out, rstd_out fp32 [T] (either may be NULL). */
 hstu_status hstu_ln_gate_fwd(const hstu_config* cfg, const void* ln_gamma, const void* ln_beta,
                              const void* o, const void* g, int64_t T, void* z_out,
                              float* mean_out, float* rstd_out, cudaStream_t stream);
 
-/* Equation (3), second half: Y = Z W2 + b2 + X.  z, x, y_out [T][d]. */
+/* Equation (3), second half: Y = Z W2 + b2 + X.  z [T][d] in cfg->dtype;
+ * x (may be NULL: no residual) and y_out [T][d] in cfg->io_dtype. */
 hstu_status hstu_proj_out_fwd(const hstu_config* cfg, const void* W2, const void* b2,
                               const void* z, const void* x, int64_t T, void* y_out,
                               cudaStream_t stream);
 
 /* Backward of hstu_proj_out_fwd: dz_out = dY W2^T; dW2 += Z^T dY; db2 += sum dY.
- * dW2/db2 may be NULL. */
+ * dy, z, dz_out in cfg->dtype.  dW2/db2 may be NULL. */
 hstu_status hstu_proj_out_bwd(const hstu_config* cfg, const void* W2, const void* z,
                               const void* dy, int64_t T, void* dz_out, float* dW2,
                               float* db2, cudaStream_t stream);
 
-/* Backward of hstu_ln_gate_fwd.  Writes dO [T][d] and, into the U columns of
+/* Backward of hstu_ln_gate_fwd (o fp32).  Writes dO [T][d] and, into the U columns of
  * dpre [T][4d], dPre_U = (dZ (.) LN(O)) (.) SiLU'(Pre_U).  Accumulates
  * dgamma, dbeta (may be NULL). */
 hstu_status hstu_ln_gate_bwd(const hstu_config* cfg, const void* ln_gamma, const void* ln_beta,
@@ -221,7 +235,8 @@ size_t hstu_attention_bwd_workspace_size(const hstu_config* cfg, int32_t B, int6
 
 /* Backward of hstu_proj_in_fwd from the assembled dPre [T][4d]:
  * dx_out = dPre W1^T + dy_resid (dy_resid may be NULL); dW1 += X^T dPre;
- * db1 += sum dPre.  dW1/db1 may be NULL. */
+ * db1 += sum dPre.  x, dpre in cfg->dtype; dy_resid, dx_out in
+ * cfg->io_dtype.  dW1/db1 may be NULL. */
 hstu_status hstu_proj_in_bwd(const hstu_config* cfg, const void* W1, const void* x,
                              const void* dpre, const void* dy_resid, int64_t T,
                              void* dx_out, float* dW1, float* db1, cudaStream_t stream);
@@ -230,7 +245,8 @@ hstu_status hstu_proj_in_bwd(const hstu_config* cfg, const void* W1, const void*
 /* Layer-level entry points (compose the steps above)                        */
 /* ------------------------------------------------------------------------ */
 
-/* One layer forward.  y [T][d].  saved: NULL for inference, else a block of
+/* One layer forward.  x, y [T][d] in cfg->io_dtype.  saved: NULL for
+ * inference, else a block of
  * hstu_workspace_size(...).saved_bytes laid out by hstu_saved_layout.
  * kv_out: NULL, or [T][2d] receiving each token's V|K (the M-FALCON history
  * cache of this layer). */
@@ -241,7 +257,8 @@ hstu_status hstu_fwd(const hstu_config* cfg, const hstu_weights* w, const void* 
                      cudaStream_t stream);
 
 /* One layer forward of M-FALCON candidates against a cached history (see
- * hstu_attention_fwd_cached for the layouts).  y [Tc][d]. */
+ * hstu_attention_fwd_cached for the layouts).  cand_x, y [Tc][d] in
+ * cfg->io_dtype; hist_kv in cfg->dtype. */
 hstu_status hstu_fwd_cached(const hstu_config* cfg, const hstu_weights* w, const void* cand_x,
                             const int64_t* cand_offsets, int32_t B, int64_t Tc,
                             const int64_t* cand_timestamps, const void* hist_kv,
@@ -250,7 +267,8 @@ hstu_status hstu_fwd_cached(const hstu_config* cfg, const hstu_weights* w, const
                             size_t ws_bytes, cudaStream_t stream);
 
 /* One layer backward.  x is the layer input of the forward, saved the block
- * the forward filled; dy [T][d] upstream; dx [T][d] output (may alias dy).
+ * the forward filled; dy [T][d] upstream; dx [T][d] output (may alias dy);
+ * x, dy, dx in cfg->io_dtype.
  * Gradients accumulate into *grads (members may be NULL). */
 hstu_status hstu_bwd(const hstu_config* cfg, const hstu_weights* w, const void* x,
                      const void* dy, const void* saved, const int64_t* seq_offsets,

@@ -360,6 +360,21 @@ hstu_status check_weights(const hstu_config* c, const hstu_weights* w, bool need
 
 namespace hstu {
 
+// Status word written by device code (bounded waits that ran out).
+__device__ uint32_t g_device_status;
+
+uint32_t* device_status() {
+  static uint32_t* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<uint32_t*>(p);
+  }
+  return ptrs[dev];
+}
+
 void prof_begin(int id, cudaStream_t s) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (!g_prof_on) return;
@@ -441,6 +456,17 @@ hstu_status hstu_profiler_collect(int32_t id, int64_t* launches, double* total_m
 }
 
 int64_t hstu_launch_count(void) { return g_launches.load(); }
+
+hstu_status hstu_device_status(uint32_t* host_out, int32_t clear, cudaStream_t stream) {
+  if (!host_out) return HSTU_ERR_INVALID;
+  uint32_t* d = device_status();
+  if (!d) return HSTU_ERR_CUDA;
+  if (cudaMemcpyAsync(host_out, d, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (clear && cudaMemsetAsync(d, 0, sizeof(uint32_t), stream) != cudaSuccess) return HSTU_ERR_CUDA;
+  return HSTU_OK;
+}
 
 hstu_status hstu_saved_layout(const hstu_config* cfg, int64_t T,
                               size_t offsets[HSTU_SAVED_COUNT + 1]) {

@@ -8,7 +8,10 @@ namespace hstu {
 cudaError_t attention_fwd_simt(int dtype, const AttnArgs& a, cudaStream_t s);
 cudaError_t attention_bwd_simt(int dtype, const AttnBwdArgs& a, cudaStream_t s);
 
-cudaError_t gemm(int dtype, const GemmArgs& g, cudaStream_t s) { return gemm_simt(dtype, g, s); }
+cudaError_t gemm(int dtype, const GemmArgs& g, cudaStream_t s) {
+  if (gemm_tc_supported(dtype, g)) return gemm_tc(g, device_status(), s);
+  return gemm_simt(dtype, g, s);
+}
 
 cudaError_t attention_fwd(int dtype, const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t s) {
   (void)ws;

@@ -1,6 +1,7 @@
 // Internal launcher interfaces shared by the .cu files of the HSTU library.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -41,6 +42,8 @@ struct GemmArgs {
 
 cudaError_t gemm(int dtype, const GemmArgs& g, cudaStream_t s);
 cudaError_t gemm_simt(int dtype, const GemmArgs& g, cudaStream_t s);
+bool gemm_tc_supported(int dtype, const GemmArgs& g);
+cudaError_t gemm_tc(const GemmArgs& g, uint32_t* status, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Attention
@@ -115,6 +118,16 @@ cudaError_t validate_inputs(const int64_t* offs, int B, int64_t T, const int64_t
 // ---------------------------------------------------------------------------
 // Launch accounting and the kernel-level profiler
 // ---------------------------------------------------------------------------
+// 2-D TMA tensor map over a row-major [outer][inner] bf16 (or fp32) array
+// with rows `row_stride_elems` apart; 128-byte swizzle unless told otherwise.
+bool encode_tmap_2d(CUtensorMap* m, bool f32, const void* ptr, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer,
+                    bool swizzle128 = true);
+
+// The library's device status word (timeouts of bounded device waits); the
+// address belongs to the current device.
+uint32_t* device_status();
+
 void prof_begin(int id, cudaStream_t s);
 void prof_end(int id, cudaStream_t s);
 void count_launch(int n = 1);

@@ -82,6 +82,7 @@ _SIGS = {
     "hstu_profiler_collect": (I32, [I32, POINTER(c_int64), POINTER(c_double)]),
     "hstu_profiler_reset": (None, []),
     "hstu_launch_count": (I64, []),
+    "hstu_device_status": (I32, [POINTER(c_uint32), I32, P]),
     "hstu_status_string": (c_char_p, [I32]),
     "hstu_version": (c_char_p, []),
 }
@@ -383,6 +384,14 @@ def profiler_collect(kernel_id: int):
 
 def launch_count() -> int:
     return int(lib().hstu_launch_count())
+
+
+def device_status(clear: bool = True, stream=None) -> int:
+    """The library's device status word (synchronises the stream)."""
+    v = c_uint32(0)
+    _check(lib().hstu_device_status(ctypes.byref(v), 1 if clear else 0, stream_ptr(stream)),
+           "hstu_device_status")
+    return v.value
 
 
 def version() -> str:

@@ -311,6 +311,14 @@ void hstu_profiler_reset(void);
  * (counted on the host whether or not the profiler is enabled). */
 int64_t hstu_launch_count(void);
 
+/* Device status word of this library on the current device: bit
+ * HSTU_DEVICE_TIMEOUT is set when a kernel's bounded wait ran out (the kernel
+ * then abandoned its work and exited cleanly; its outputs are not valid).
+ * Copies the word to *host_out, synchronising `stream`; clears it when
+ * `clear` is non-zero. */
+#define HSTU_DEVICE_TIMEOUT 0x100u
+hstu_status hstu_device_status(uint32_t* host_out, int32_t clear, cudaStream_t stream);
+
 const char* hstu_status_string(hstu_status s);
 const char* hstu_version(void);
 

@@ -14,7 +14,12 @@ were each rounded to bf16 a few times; that noise has a relative std of about
 2^-9 per rounding, so the normwise error is a fraction of a percent while the
 largest of the ~10^6 entries sits about 5 standard deviations out.  They are
 checked normwise and entry-wise:
-    ||gpu - oracle||_2 / ||oracle||_2 <= tol / 2,  max |gpu - oracle| <= 3 tol rms(oracle).
+    ||gpu - oracle||_2 / ||oracle||_2 <= tol / 2
+    max_i |gpu_i - oracle_i| / (rms(oracle) + |oracle_i|) <= 3 tol
+(for noise of uniform size the largest of M entries is about sqrt(2 ln 2M),
+i.e. 5 to 6 for M ~ 1e6, times the normwise level; entries that are sums of
+many more terms, like the rab bucket that collects all distant pairs, carry
+noise in proportion to their size, hence the |oracle_i| term).
 The oracle consumes the exact (bf16-rounded) inputs the GPU sees, in fp64.
 """
 import numpy as np
@@ -70,13 +75,14 @@ def check_el(got, ref, dtype, what, scale=1.0):
 
 
 def check_grad(got, ref, dtype, what):
-    """Parameter gradients: normwise <= tol/2 and max entry <= 3 tol rms."""
+    """Parameter gradients: normwise <= tol/2 and entry-wise
+    |err_i| / (rms + |ref_i|) <= 3 tol."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape and np.isfinite(got).all(), what
     nrm = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
     assert nrm <= TOL[dtype] / 2, f"{what}: normwise {nrm:.3e} > {TOL[dtype] / 2:.1e}"
-    check(got, ref, dtype, what, scale=3.0)
+    check_el(got, ref, dtype, what, scale=3.0)
     return nrm
 
 

@@ -160,8 +160,8 @@ hstu_status do_proj_in(const hstu_config* c, const void* W1, const void* b1, con
 }
 
 AttnArgs full_attn_args(const hstu_config* c, const float* rp, const float* rt, const void* g,
-                        const int64_t* offs, int B, const int64_t* ts, const int32_t* nt,
-                        void* o) {
+                        const int64_t* offs, int B, int64_t T, const int64_t* ts,
+                        const int32_t* nt, void* o) {
   const int d = c->d_model, es = dtype_size(c->dtype);
   AttnArgs a;
   a.q = at(const_cast<void*>(g), (size_t)2 * d * es);
@@ -185,6 +185,8 @@ AttnArgs full_attn_args(const hstu_config* c, const float* rp, const float* rt, 
   a.P = c->num_pos_buckets;
   a.Bt = c->num_time_buckets;
   a.max_q_len = c->max_seq_len;
+  a.q_rows = T;
+  a.kv_rows = T;
   a.rab_pos = rp;
   a.rab_time = rt;
   a.inv_N = 1.0f / c->norm_N;
@@ -267,7 +269,7 @@ hstu_status do_attention_bwd(const hstu_config* c, const float* rp, const float*
                              cudaStream_t s) {
   const int d = c->d_model, es = dtype_size(c->dtype);
   AttnBwdArgs a;
-  a.f = full_attn_args(c, rp, rt, g, offs, B, ts, nt, nullptr);
+  a.f = full_attn_args(c, rp, rt, g, offs, B, T, ts, nt, nullptr);
   a.dout = dO;
   a.pre = pre;
   a.dpre = dpre;
@@ -543,8 +545,8 @@ hstu_status hstu_attention_fwd(const hstu_config* cfg, const float* rab_pos, con
   if (ws_bytes < need_ws) return HSTU_ERR_WORKSPACE;
   if (need_ws > 0) HSTU_TRY(need(workspace, 1));
   if (T == 0 || B == 0) return HSTU_OK;
-  AttnArgs a = full_attn_args(cfg, rab_pos, rab_time, g, seq_offsets, B, timestamps, num_targets,
-                              o_out);
+  AttnArgs a = full_attn_args(cfg, rab_pos, rab_time, g, seq_offsets, B, T, timestamps,
+                              num_targets, o_out);
   return do_attention_fwd(cfg, a, workspace, ws_bytes, stream, HSTU_K_ATTN_FWD);
 }
 
@@ -568,9 +570,10 @@ hstu_status hstu_attention_fwd_cached(const hstu_config* cfg, const float* rab_p
   if (need_ws > 0) HSTU_TRY(need(workspace, 1));
   if (Tc == 0 || B == 0) return HSTU_OK;
   const int d = cfg->d_model, es = dtype_size(cfg->dtype);
-  AttnArgs a = full_attn_args(cfg, rab_pos, rab_time, cand_g, cand_offsets, B, cand_timestamps,
-                              nullptr, o_out);
+  AttnArgs a = full_attn_args(cfg, rab_pos, rab_time, cand_g, cand_offsets, B, Tc,
+                              cand_timestamps, nullptr, o_out);
   a.cached = 1;
+  a.kv_rows = T_hist;
   a.v = hist_kv;
   a.k = at(const_cast<void*>(hist_kv), (size_t)d * es);
   a.kv_stride = 2 * d;
@@ -727,7 +730,7 @@ hstu_status hstu_fwd(const hstu_config* cfg, const hstu_weights* w, const void* 
   const void* xop = nullptr;
   HSTU_TRY(to_operand(cfg, x, T, xlow, &xop, stream));
   HSTU_TRY(do_proj_in(cfg, w->W1, w->b1, xop, T, pre, g, stream));
-  AttnArgs a = full_attn_args(cfg, w->rab_pos, w->rab_time, g, seq_offsets, B, timestamps,
+  AttnArgs a = full_attn_args(cfg, w->rab_pos, w->rab_time, g, seq_offsets, B, T, timestamps,
                               num_targets, o);
   HSTU_TRY(do_attention_fwd(cfg, a, at(workspace, L.attn), ws_bytes - L.attn, stream,
                             HSTU_K_ATTN_FWD));
@@ -770,9 +773,10 @@ hstu_status hstu_fwd_cached(const hstu_config* cfg, const hstu_weights* w, const
   const void* xop = nullptr;
   HSTU_TRY(to_operand(cfg, cand_x, Tc, at(workspace, L.xlow), &xop, stream));
   HSTU_TRY(do_proj_in(cfg, w->W1, w->b1, xop, Tc, nullptr, g, stream));
-  AttnArgs a = full_attn_args(cfg, w->rab_pos, w->rab_time, g, cand_offsets, B, cand_timestamps,
-                              nullptr, o);
+  AttnArgs a = full_attn_args(cfg, w->rab_pos, w->rab_time, g, cand_offsets, B, Tc,
+                              cand_timestamps, nullptr, o);
   a.cached = 1;
+  a.kv_rows = T_hist;
   a.v = hist_kv;
   a.k = at(const_cast<void*>(hist_kv), (size_t)d * es);
   a.kv_stride = 2 * d;

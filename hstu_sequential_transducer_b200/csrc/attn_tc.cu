@@ -1,0 +1,565 @@
+// Tensor-core (tcgen05) pointwise aggregated attention, forward.
+//
+// Equation (2) of the HSTU walkthrough ("What an HSTU layer changes"):
+//   O_h = (1/N) [M (.) SiLU(Q_h K_h^T + rab^{p,t}_h)] V_h
+// with no softmax ("No sequence-wise softmax"), rab^{p,t} from relative
+// position and elapsed time (course notes, "Problem 2"), the causal or
+// M-FALCON target mask ("What HSTU actually changed") and ragged work
+// ("Ragged kernels"): only the key tiles a query tile can see are visited.
+//
+// Work items are (sequence, head, 128-row query tile), ordered longest-first
+// by a device-side counting sort (attn_sched) and dealt round-robin to one
+// persistent CTA per SM.  Per CTA:
+//   warp 0      TMA producer: Q tile once per item; K and V tiles (128 keys) and
+//               the keys' timestamps into a ring of stages
+//   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S
+//               buffers; O += P V with P read from TMEM (A operand in TMEM)
+//   warps 2..5  one query row per thread: S from TMEM, bucketed rab bias, mask,
+//               SiLU, P (bf16) written back over S; at the end of an item, O
+//               from TMEM times 1/N plus the candidates' self term, to HBM
+// tcgen05.mma instructions of one thread execute in issue order, so the QK^T
+// of tile j+2 overwrites S/P buffer j%2 only after the PV of tile j read it.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace hstu {
+
+using namespace tc;
+
+// ---------------------------------------------------------------------------
+// Work list: items sorted by descending number of key tiles
+// ---------------------------------------------------------------------------
+struct AttnItem {
+  int32_t b;
+  int16_t qt;
+  int16_t h;
+};
+
+constexpr int kTile = 128;
+constexpr int kMaxCost = 514;  // key tiles per item, 65536 / 128 + 2
+
+struct SchedWs {
+  int32_t* hist;     // [kMaxCost]
+  int32_t* cursor;   // [kMaxCost]
+  int32_t* total;    // [1]
+  AttnItem* items;   // [max_items]
+};
+
+size_t attn_sched_bytes(int B, int64_t Tq, int H) {
+  const size_t max_items = ((size_t)(Tq / kTile) + (size_t)B + 1) * (size_t)H;
+  return align_up(3 * kMaxCost * sizeof(int32_t), 256) + max_items * sizeof(AttnItem);
+}
+
+SchedWs sched_ws(void* ws) {
+  SchedWs s;
+  s.hist = static_cast<int32_t*>(ws);
+  s.cursor = s.hist + kMaxCost;
+  s.total = s.cursor + kMaxCost;
+  s.items = reinterpret_cast<AttnItem*>(static_cast<char*>(ws) + align_up(3 * kMaxCost * sizeof(int32_t), 256));
+  return s;
+}
+
+// Key tiles an item needs, and the item's geometry.
+struct SeqGeom {
+  int64_t qs, ks;   // first query row, first key row
+  int nq, hlen;     // queries; keys visible to candidates (= history length)
+  int qbase;        // position of query 0
+};
+
+__device__ __forceinline__ SeqGeom seq_geom(const AttnArgs& a, int b) {
+  SeqGeom g;
+  g.qs = a.q_offsets[b];
+  g.nq = (int)(a.q_offsets[b + 1] - g.qs);
+  g.ks = a.kv_offsets[b];
+  const int nkv = (int)(a.kv_offsets[b + 1] - g.ks);
+  if (a.cached) {
+    g.hlen = nkv;
+    g.qbase = nkv;
+  } else {
+    const int m = a.num_targets ? a.num_targets[b] : 0;
+    g.hlen = min(max(g.nq - m, 0), g.nq);
+    g.qbase = 0;
+  }
+  return g;
+}
+
+__device__ __forceinline__ int item_kend(const SeqGeom& g, int qt) {
+  const int rows = min(kTile, g.nq - qt * kTile);
+  return min(g.hlen, g.qbase + qt * kTile + rows);
+}
+
+__global__ void sched_count_kernel(AttnArgs a, SchedWs w) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < a.B; b += gridDim.x * blockDim.x) {
+    const SeqGeom g = seq_geom(a, b);
+    const int ntile = (g.nq + kTile - 1) / kTile;
+    for (int qt = 0; qt < ntile; ++qt) {
+      const int cost = min((item_kend(g, qt) + kTile - 1) / kTile, kMaxCost - 1);
+      atomicAdd(&w.hist[cost], a.H);
+    }
+  }
+}
+
+// One warp: cursor[c] = number of items of cost > c (descending order).
+__global__ void sched_scan_kernel(SchedWs w) {
+  if (threadIdx.x != 0) return;
+  int run = 0;
+  for (int c = kMaxCost - 1; c >= 0; --c) {
+    w.cursor[c] = run;
+    run += w.hist[c];
+  }
+  *w.total = run;
+}
+
+__global__ void sched_fill_kernel(AttnArgs a, SchedWs w) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < a.B; b += gridDim.x * blockDim.x) {
+    const SeqGeom g = seq_geom(a, b);
+    const int ntile = (g.nq + kTile - 1) / kTile;
+    for (int qt = 0; qt < ntile; ++qt) {
+      const int cost = min((item_kend(g, qt) + kTile - 1) / kTile, kMaxCost - 1);
+      const int pos = atomicAdd(&w.cursor[cost], a.H);
+      for (int h = 0; h < a.H; ++h) {
+        AttnItem it;
+        it.b = b;
+        it.qt = (int16_t)qt;
+        it.h = (int16_t)h;
+        w.items[pos + h] = it;
+      }
+    }
+  }
+}
+
+cudaError_t build_schedule(const AttnArgs& a, void* ws, cudaStream_t s) {
+  SchedWs w = sched_ws(ws);
+  cudaError_t e = cudaMemsetAsync(w.hist, 0, 3 * kMaxCost * sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
+  const int blocks = (a.B + 255) / 256;
+  sched_count_kernel<<<blocks, 256, 0, s>>>(a, w);
+  sched_scan_kernel<<<1, 32, 0, s>>>(w);
+  sched_fill_kernel<<<blocks, 256, 0, s>>>(a, w);
+  count_launch(3);
+  return cudaGetLastError();
+}
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// The forward kernel
+// ---------------------------------------------------------------------------
+template <int DH>
+struct FwdCfg {
+  static constexpr int BOXES = DH / 64;                 // 64-column boxes per tile row
+  static constexpr int TILE_BYTES = kTile * DH * 2;     // one 128 x DH bf16 tile
+  static constexpr int STAGES = 2;
+  static constexpr int KV_BYTES = 2 * TILE_BYTES;       // K and V
+  static constexpr int TS_BYTES = kTile * 8;            // key timestamps
+  static constexpr int STAGE_BYTES = KV_BYTES + TS_BYTES;
+  static constexpr int SMEM_USED = 1024 + TILE_BYTES + STAGES * STAGE_BYTES + 1024;
+  // at least half of the SM's shared memory, so that one CTA (and its 512
+  // TMEM columns) is resident per SM
+  static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, kTile, false, false);
+  static constexpr uint32_t IDESC_O = idesc_bf16(128, DH, false, true);
+  static constexpr uint32_t TMEM_COLS = 512;            // S0, S1, O
+};
+
+struct FwdParams {
+  AttnArgs a;
+  SchedWs w;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ float silu_fast(float x) {
+  // x * sigmoid(x) = h + h * tanh(h) with h = x / 2
+  const float h = 0.5f * x;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
+
+template <int DH>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const FwdParams P) {
+  using C = FwdCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sStage = sQ + C::TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + C::STAGES * C::STAGE_BYTES);
+  uint64_t* q_full = bars;                   // 1
+  uint64_t* q_empty = bars + 1;              // 1
+  uint64_t* kv_full = bars + 2;              // STAGES
+  uint64_t* kv_empty = kv_full + C::STAGES;  // STAGES
+  uint64_t* s_full = kv_empty + C::STAGES;   // 2
+  uint64_t* p_full = s_full + 2;             // 2
+  uint64_t* o_full = p_full + 2;             // 1
+  uint64_t* o_free = o_full + 1;             // 1
+  uint64_t* done_bar = o_free + 1;           // 1
+  float* rab = reinterpret_cast<float*>(done_bar + 1);   // [2][32] of the current head
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rab + 64);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const AttnArgs& a = P.a;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int total = *P.w.total;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+    }
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 4);
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO = tmem + 256;
+
+  // Every role walks the same item sequence and numbers the key tiles it
+  // meets with one running counter n: K/V stage n % STAGES (parity
+  // (n / STAGES) & 1) and S/P buffer n & 1 (parity (n >> 1) & 1).
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t n = 0, items_done = 0;
+    uint32_t issued = 0, issued_par = 0;
+    bool q_issued = false;
+    uint32_t q_par = 0;
+    for (int it = blockIdx.x; it < total; it += gridDim.x) {
+      if (*abort_flag) break;
+      const AttnItem item = P.w.items[it];
+      const SeqGeom g = seq_geom(a, item.b);
+      const int r0 = item.qt * kTile;
+      const int kend = item_kend(g, item.qt);
+      const int nk = (kend + kTile - 1) / kTile;
+      if (nk == 0) continue;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(q_empty, (items_done & 1) ^ 1, abort_flag, P.status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_expect_tx(q_full, C::TILE_BYTES);
+#pragma unroll
+        for (int x = 0; x < C::BOXES; ++x)
+          tma_load_2d(sQ + x * (kTile * 128), &tmQ, q_full, item.h * DH + 64 * x, (int32_t)(g.qs + r0));
+        q_issued = true;
+        q_par = items_done & 1;
+      }
+      ++items_done;
+      for (int j = 0; j < nk; ++j, ++n) {
+        const int stage = (int)(n % C::STAGES);
+        const uint32_t par = (n / C::STAGES) & 1;
+        if (lane == 0) ok = mbar_wait(&kv_empty[stage], par ^ 1, abort_flag, P.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        uint8_t* st = sStage + stage * C::STAGE_BYTES;
+        long long* kts = reinterpret_cast<long long*>(st + C::KV_BYTES);
+        const int k0 = j * kTile;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = lane + 32 * q;
+          kts[c] = (k0 + c < kend) ? a.kv_ts[g.ks + k0 + c] : 0;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_expect_tx(&kv_full[stage], C::KV_BYTES);
+#pragma unroll
+          for (int x = 0; x < C::BOXES; ++x) {
+            tma_load_2d(st + x * (kTile * 128), &tmK, &kv_full[stage], item.h * DH + 64 * x,
+                        (int32_t)(g.ks + k0));
+            tma_load_2d(st + C::TILE_BYTES + x * (kTile * 128), &tmV, &kv_full[stage],
+                        item.h * DH + 64 * x, (int32_t)(g.ks + k0));
+          }
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (par << stage);
+        }
+      }
+      if (!ok) break;
+    }
+    if (lane == 0) {
+      volatile int never = 0;
+      for (int s2 = 0; s2 < C::STAGES; ++s2)
+        if (issued & (1u << s2)) mbar_wait(&kv_full[s2], (issued_par >> s2) & 1u, &never, P.status);
+      if (q_issued) mbar_wait(q_full, q_par, &never, P.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t n = 0, items_done = 0;
+      for (int it = blockIdx.x; it < total; it += gridDim.x) {
+        if (*abort_flag) break;
+        const AttnItem item = P.w.items[it];
+        const SeqGeom g = seq_geom(a, item.b);
+        const int kend = item_kend(g, item.qt);
+        const int nk = (kend + kTile - 1) / kTile;
+        if (nk == 0) continue;
+        if (!mbar_wait(q_full, items_done & 1, abort_flag, P.status)) break;
+        if (!mbar_wait(o_free, (items_done & 1) ^ 1, abort_flag, P.status)) break;
+        tc_fence_after();
+        const uint32_t q0 = smem_u32(sQ);
+        bool ok = true;
+        for (int j = 0; j <= nk; ++j) {
+          if (j < nk) {
+            // S_j = Q K_j^T into buffer (n + j) & 1
+            const uint32_t nj = n + j;
+            const int stage = (int)(nj % C::STAGES);
+            if (!mbar_wait(&kv_full[stage], (nj / C::STAGES) & 1, abort_flag, P.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t k0s = smem_u32(sStage + stage * C::STAGE_BYTES);
+#pragma unroll
+            for (int k = 0; k < DH / 16; ++k) {
+              const uint32_t off = (k / 4) * (kTile * 128) + (k % 4) * 32;
+              mma_ss(tS[nj & 1], sdesc_kmajor(q0 + off), sdesc_kmajor(k0s + off), C::IDESC_S, k > 0);
+            }
+            mma_commit(&s_full[nj & 1]);
+            if (j == nk - 1) mma_commit(q_empty);
+          }
+          if (j >= 1) {
+            // O += P_{j-1} V_{j-1}
+            const uint32_t np = n + j - 1;
+            if (!mbar_wait(&p_full[np & 1], (np >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            tc_fence_after();
+            const int pst = (int)(np % C::STAGES);
+            const uint32_t v0 = smem_u32(sStage + pst * C::STAGE_BYTES) + C::TILE_BYTES;
+#pragma unroll
+            for (int k = 0; k < kTile / 16; ++k)
+              mma_ts(tO, tS[np & 1] + k * 8, sdesc_mnmajor(v0 + k * 2048, kTile * 128), C::IDESC_O,
+                     (j > 1 || k > 0) ? 1u : 0u);
+            mma_commit(&kv_empty[pst]);
+          }
+        }
+        if (!ok) break;
+        n += nk;
+        ++items_done;
+        mma_commit(o_full);
+      }
+      mma_commit(done_bar);
+      volatile int never = 0;
+      mbar_wait(done_bar, 0, &never, P.status);
+    }
+  } else {
+    // ------------------------------------------------------------ activation + epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    uint32_t n = 0, items_done = 0;
+    int cur_h = -1;
+    for (int it = blockIdx.x; it < total; it += gridDim.x) {
+      const AttnItem item = P.w.items[it];
+      const SeqGeom g = seq_geom(a, item.b);
+      const int r0 = item.qt * kTile;
+      const int rows = min(kTile, g.nq - r0);
+      const int kend = item_kend(g, item.qt);
+      const int nk = (kend + kTile - 1) / kTile;
+      const bool rvalid = row < rows;
+      const int qpos = g.qbase + r0 + row;
+      const int qp_clamped = min(qpos, g.hlen);
+      const bool cand = qpos >= g.hlen;
+      const long long tq = rvalid ? a.q_ts[g.qs + r0 + row] : 0;
+      if (item.h != cur_h) {
+        named_barrier(1, 128);
+        if (row < 32) {
+          rab[row] = (a.rab_pos && row < a.P) ? a.rab_pos[item.h * a.P + row] : 0.f;
+          rab[32 + row] = (a.rab_time && row < a.Bt) ? a.rab_time[item.h * a.Bt + row] : 0.f;
+        }
+        named_barrier(1, 128);
+        cur_h = item.h;
+      }
+      bool stop = *abort_flag != 0;
+      if (named_barrier_any(1, 128, stop)) break;
+      bool fail = false;
+      for (int j = 0; j < nk; ++j) {
+        const uint32_t nj = n + j;
+        const uint32_t buf = nj & 1, par = (nj >> 1) & 1;
+        fail = !mbar_wait(&s_full[buf], par, abort_flag, P.status);
+        if (named_barrier_any(1, 128, fail)) { fail = true; break; }
+        tc_fence_after();
+        // the stage holding this tile's keys (and their timestamps)
+        const int kst = (int)(nj % C::STAGES);
+        const long long* kts = reinterpret_cast<const long long*>(sStage + kst * C::STAGE_BYTES + C::KV_BYTES);
+        const int k0 = j * kTile;
+        const bool need_mask = (k0 + kTile > kend) || (!cand && k0 + kTile - 1 > qpos) || !rvalid;
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t s[32];
+          tmem_ld32(tS[buf] + lane_off + c * 32, s);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int col = c * 32 + e + u;
+              const int jk = k0 + col;
+              const int dp = qp_clamped - jk;
+              const int bp = min(max(dp, 0), a.P - 1);
+              const long long dt = tq - kts[col];
+              const int bt = dt <= 0 ? 0 : min(64 - __clzll(dt), a.Bt - 1);
+              float x = __uint_as_float(s[e + u]) + rab[bp] + rab[32 + bt];
+              float y = silu_fast(x);
+              if (need_mask) {
+                const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
+                y = ok ? y : 0.f;
+              }
+              pv[u] = y;
+            }
+            pk[e / 2] = pack_bf16(pv[0], pv[1]);
+          }
+          tmem_st16(tS[buf] + lane_off + c * 16, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[buf]);
+      }
+      if (fail) break;
+      n += nk;
+      // ---- epilogue: O (fp32) = (1/N) (P V  [+ self term])
+      float* O = static_cast<float*>(a.o);
+      const int h = item.h;
+      float self_w = 0.f;
+      if (cand && rvalid) {
+        const bf16* q = static_cast<const bf16*>(a.q) + (g.qs + r0 + row) * a.q_stride + h * DH;
+        const bf16* k = static_cast<const bf16*>(a.self_k) + (g.qs + r0 + row) * a.q_stride + h * DH;
+        float sdot = 0.f;
+#pragma unroll 4
+        for (int e = 0; e < DH; e += 8) {
+          const uint4 qa = *reinterpret_cast<const uint4*>(q + e);
+          const uint4 ka = *reinterpret_cast<const uint4*>(k + e);
+          const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qa);
+          const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&ka);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 qf = __bfloat1622float2(qh[u]), kf = __bfloat1622float2(kh[u]);
+            sdot = fmaf(qf.x, kf.x, sdot);
+            sdot = fmaf(qf.y, kf.y, sdot);
+          }
+        }
+        self_w = silu_acc(sdot + rab[0] + rab[32]);
+      }
+      if (nk > 0) {
+        fail = !mbar_wait(o_full, items_done & 1, abort_flag, P.status);
+        ++items_done;
+        if (named_barrier_any(1, 128, fail)) break;
+        tc_fence_after();
+      }
+      const bf16* sv = static_cast<const bf16*>(a.self_v) + (g.qs + r0 + row) * a.q_stride + h * DH;
+#pragma unroll
+      for (int c = 0; c < DH / 32; ++c) {
+        float o[32];
+        if (nk > 0) {
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(r[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+        if (rvalid) {
+          if (cand) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              const uint4 va = *reinterpret_cast<const uint4*>(sv + c * 32 + i);
+              const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&va);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 vf = __bfloat1622float2(vh[u]);
+                o[i + 2 * u] = fmaf(self_w, vf.x, o[i + 2 * u]);
+                o[i + 2 * u + 1] = fmaf(self_w, vf.y, o[i + 2 * u + 1]);
+              }
+            }
+          }
+          float* dst = O + (g.qs + r0 + row) * a.o_stride + h * DH + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(o[i] * a.inv_N, o[i + 1] * a.inv_N, o[i + 2] * a.inv_N, o[i + 3] * a.inv_N);
+        }
+      }
+      if (nk > 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_free);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+int sm_count_attn() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int DH>
+cudaError_t launch_fwd(const AttnArgs& a, void* ws, uint32_t* status, cudaStream_t s) {
+  using C = FwdCfg<DH>;
+  // Tensor maps over the Q block of the query rows' G and the K and V blocks
+  // of the key rows: each starts at its block's head-0 column, d columns wide,
+  // rows q_stride / kv_stride elements apart; a box is 64 columns x 128 rows.
+  const int d = a.H * DH;
+  CUtensorMap tQ, tK, tV;
+  const bf16* q = static_cast<const bf16*>(a.q);
+  const bf16* k = static_cast<const bf16*>(a.k);
+  const bf16* v = static_cast<const bf16*>(a.v);
+  FwdParams P;
+  P.a = a;
+  P.w = sched_ws(ws);
+  P.status = status;
+  bool ok = encode_tmap_2d(&tQ, false, q, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)a.q_stride, 64, kTile) &&
+            encode_tmap_2d(&tK, false, k, (uint64_t)d, (uint64_t)a.kv_rows, (uint64_t)a.kv_stride, 64, kTile) &&
+            encode_tmap_2d(&tV, false, v, (uint64_t)d, (uint64_t)a.kv_rows, (uint64_t)a.kv_stride, 64, kTile);
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = build_schedule(a, ws, s);
+  if (e != cudaSuccess) return e;
+  auto kern = attn_fwd_tc_kernel<DH>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<sm_count_attn(), 192, C::SMEM, s>>>(tQ, tK, tV, P);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attention_fwd_tc_supported(int dtype, const AttnArgs& a) {
+  return dtype == HSTU_BF16 && (a.dh == 64 || a.dh == 128) && a.q_rows > 0 && a.kv_rows > 0 &&
+         a.q_stride % 8 == 0 && a.kv_stride % 8 == 0 && a.P <= 32 && a.Bt <= 32;
+}
+
+cudaError_t attention_fwd_tc(const AttnArgs& a, void* ws, uint32_t* status, cudaStream_t s) {
+  if (a.dh == 128) return launch_fwd<128>(a, ws, status, s);
+  return launch_fwd<64>(a, ws, status, s);
+}
+
+}  // namespace hstu

@@ -14,8 +14,9 @@ cudaError_t gemm(int dtype, const GemmArgs& g, cudaStream_t s) {
 }
 
 cudaError_t attention_fwd(int dtype, const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t s) {
-  (void)ws;
-  (void)ws_bytes;
+  if (attention_fwd_tc_supported(dtype, a) &&
+      ws_bytes >= attn_sched_bytes(a.B, a.q_rows, a.H))
+    return attention_fwd_tc(a, ws, device_status(), s);
   return attention_fwd_simt(dtype, a, s);
 }
 
@@ -27,8 +28,8 @@ cudaError_t attention_bwd(int dtype, const AttnBwdArgs& a, void* ws, size_t ws_b
 }
 
 size_t attention_fwd_ws(int B, int64_t T, int H, int max_len) {
-  (void)B; (void)T; (void)H; (void)max_len;
-  return 0;
+  (void)max_len;
+  return attn_sched_bytes(B, T, H);
 }
 size_t attention_bwd_ws(int B, int64_t T, int H, int d, int max_len) {
   (void)B; (void)T; (void)H; (void)d; (void)max_len;

@@ -68,6 +68,8 @@ struct AttnArgs {
   int cached = 0;                // 0: queries and keys are the same sequence; 1: M-FALCON cache
   int B = 0, H = 0, dh = 0, P = 32, Bt = 32;
   int max_q_len = 0;             // upper bound of any query sequence length
+  int64_t q_rows = 0;            // rows of the query-side tensor (T or Tc)
+  int64_t kv_rows = 0;           // rows of the key-side tensor (T or T_hist)
   const float* rab_pos = nullptr;
   const float* rab_time = nullptr;
   float inv_N = 1.0f;
@@ -89,6 +91,9 @@ cudaError_t attention_fwd(int dtype, const AttnArgs& a, void* ws, size_t ws_byte
 cudaError_t attention_bwd(int dtype, const AttnBwdArgs& a, void* ws, size_t ws_bytes,
                           cudaStream_t s);
 size_t attention_fwd_ws(int B, int64_t T, int H, int max_len);
+size_t attn_sched_bytes(int B, int64_t Tq, int H);
+bool attention_fwd_tc_supported(int dtype, const AttnArgs& a);
+cudaError_t attention_fwd_tc(const AttnArgs& a, void* ws, uint32_t* status, cudaStream_t s);
 size_t attention_bwd_ws(int B, int64_t T, int H, int d, int max_len);
 
 // ---------------------------------------------------------------------------

@@ -1,0 +1,570 @@
+// Tensor-core (tcgen05) pointwise-attention backward.
+//
+// For every allowed pair (i query, j key) of equation (2) of the HSTU
+// walkthrough, with S = q_i.k_j + rab and A = SiLU(S)/N:
+//   dA = dO_i . v_j,   dS = dA SiLU'(S) / N
+//   dV_j += A dO_i,  dK_j += dS q_i,  dQ_i += dS k_j,  drab[bucket] += dS
+// There is no softmax, so nothing needs row statistics: dS is elementwise.
+//
+// Work items are (sequence, head, 128-key tile of the history), ordered by
+// descending number of query tiles and dealt round-robin to one persistent
+// CTA per SM.  Per item the key tile's K and V stay in shared memory and the
+// CTA walks the query tiles that see it (causal: from the key tile on;
+// candidates see every history key):
+//   warp 0      TMA producer: K, V once per item; Q_i, dO_i and the queries'
+//               timestamps per query tile
+//   warp 1      MMA issuer: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM; then
+//               dV += P^T dO_i and dK += dS^T Q_i (P^T, dS^T as TMEM A
+//               operands) and dQ_i = dS K (dS from shared memory)
+//   warps 2..5  one key row per thread: P^T and dS^T from S^T, dP^T; dS into
+//               shared memory; run-length sums of dS per rab bucket; then dQ_i
+//               from TMEM into the fp32 dQ accumulator (vector reductions);
+//               after the last query tile dK, dV times SiLU'(Pre) to dPre
+// TMEM (512 columns): [0,128) S^T -> P^T -> dQ_i, [128,256) dP^T -> dS^T,
+// [256,384) dV, [384,512) dK.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace hstu {
+
+using namespace tc;
+
+namespace {
+
+constexpr int kT = 128;
+constexpr int kMaxCostB = 514;
+
+struct BItem {
+  int32_t b;
+  int16_t kt;
+  int16_t h;
+};
+
+struct BSched {
+  int32_t* hist;
+  int32_t* cursor;
+  int32_t* total;
+  BItem* items;
+};
+
+BSched bsched(void* ws) {
+  BSched s;
+  s.hist = static_cast<int32_t*>(ws);
+  s.cursor = s.hist + kMaxCostB;
+  s.total = s.cursor + kMaxCostB;
+  s.items = reinterpret_cast<BItem*>(static_cast<char*>(ws) + align_up(3 * kMaxCostB * sizeof(int32_t), 256));
+  return s;
+}
+
+__device__ __forceinline__ void bgeom(const AttnArgs& a, int b, int64_t& s0, int& n, int& hlen) {
+  s0 = a.q_offsets[b];
+  n = (int)(a.q_offsets[b + 1] - s0);
+  const int m = a.num_targets ? a.num_targets[b] : 0;
+  hlen = min(max(n - m, 0), n);
+}
+
+// query tiles that see key tile kt: from kt (causal) to the end
+__device__ __forceinline__ int bcost(int n, int kt) { return (n + kT - 1) / kT - kt; }
+
+__global__ void bsched_count(AttnArgs a, BSched w) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < a.B; b += gridDim.x * blockDim.x) {
+    int64_t s0;
+    int n, hlen;
+    bgeom(a, b, s0, n, hlen);
+    for (int kt = 0; kt * kT < hlen; ++kt)
+      atomicAdd(&w.hist[min(bcost(n, kt), kMaxCostB - 1)], a.H);
+  }
+}
+__global__ void bsched_scan(BSched w) {
+  if (threadIdx.x != 0) return;
+  int run = 0;
+  for (int c = kMaxCostB - 1; c >= 0; --c) {
+    w.cursor[c] = run;
+    run += w.hist[c];
+  }
+  *w.total = run;
+}
+__global__ void bsched_fill(AttnArgs a, BSched w) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < a.B; b += gridDim.x * blockDim.x) {
+    int64_t s0;
+    int n, hlen;
+    bgeom(a, b, s0, n, hlen);
+    for (int kt = 0; kt * kT < hlen; ++kt) {
+      const int pos = atomicAdd(&w.cursor[min(bcost(n, kt), kMaxCostB - 1)], a.H);
+      for (int h = 0; h < a.H; ++h) {
+        BItem it;
+        it.b = b;
+        it.kt = (int16_t)kt;
+        it.h = (int16_t)h;
+        w.items[pos + h] = it;
+      }
+    }
+  }
+}
+
+template <int DH>
+struct BCfg {
+  static constexpr int BOXES = DH / 64;
+  static constexpr int TILE = kT * DH * 2;          // 128 rows x DH bf16
+  static constexpr int QD_BYTES = 2 * TILE;         // Q_i and dO_i
+  static constexpr int TS_BYTES = kT * 8;
+  static constexpr int STAGE = QD_BYTES + TS_BYTES;
+  static constexpr int DS_BYTES = kT * kT * 2;      // dS [key][query] bf16
+  static constexpr int SMEM_USED = 1024 + 2 * TILE + STAGE + DS_BYTES + 2048;
+  // at least half of the SM's shared memory: one CTA (512 TMEM columns) per SM
+  static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static constexpr uint32_t IDESC_ST = idesc_bf16(128, kT, false, false);   // K Q^T, V dO^T
+  static constexpr uint32_t IDESC_DKV = idesc_bf16(128, DH, false, true);   // P^T dO, dS^T Q
+  static constexpr uint32_t IDESC_DQ = idesc_bf16(128, DH, true, true);     // dS K
+};
+
+struct BParams {
+  AttnBwdArgs A;
+  BSched w;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ float tanh_fast(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
+  return t;
+}
+
+// Byte offset of (row k, column c) in a 128-byte-swizzled MN-major tile whose
+// MN extent (c) is split into 64-wide blocks `blk` bytes apart and whose K
+// extent (k) runs down 128-byte rows.
+__device__ __forceinline__ uint32_t mn_off(int k, int c, uint32_t blk) {
+  return (uint32_t)(c >> 6) * blk + (uint32_t)(k >> 3) * 1024u + (uint32_t)(k & 7) * 128u +
+         ((uint32_t)(((c & 63) >> 3) ^ (k & 7)) << 4) + (uint32_t)(c & 7) * 2u;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                       const BParams P) {
+  using C = BCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + C::TILE;
+  uint8_t* sQD = sV + C::TILE;        // Q_i | dO_i | query timestamps
+  uint8_t* sDS = sQD + C::STAGE;      // dS, MN-major for the dQ MMA
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + C::DS_BYTES);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* qd_full = bars + 2;
+  uint64_t* qd_empty = bars + 3;
+  uint64_t* st_full = bars + 4;
+  uint64_t* pds_full = bars + 5;
+  uint64_t* dq_full = bars + 6;
+  uint64_t* a_free = bars + 7;
+  uint64_t* dkv_full = bars + 8;
+  uint64_t* dkv_free = bars + 9;
+  uint64_t* done_bar = bars + 10;
+  float* rab = reinterpret_cast<float*>(bars + 12);     // [64] current head's tables
+  float* drab = rab + 64;                               // [64] bucket sums of dS
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drab + 64);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const AttnArgs& a = P.A.f;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int total = *P.w.total;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 11; ++i) {
+      const bool four = &bars[i] == pds_full || &bars[i] == a_free || &bars[i] == dkv_free;
+      mbar_init(&bars[i], four ? 4 : 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tA = tmem, tB = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t items_done = 0, m = 0;
+    bool kv_iss = false, qd_iss = false;
+    uint32_t kv_par = 0, qd_par = 0;
+    for (int it = blockIdx.x; it < total; it += gridDim.x) {
+      if (*abort_flag) break;
+      const BItem item = P.w.items[it];
+      int64_t s0;
+      int n, hlen;
+      bgeom(a, item.b, s0, n, hlen);
+      const int k0 = item.kt * kT;
+      const int nqt = bcost(n, item.kt);
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(kv_empty, (items_done & 1) ^ 1, abort_flag, P.status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_expect_tx(kv_full, 2 * C::TILE);
+#pragma unroll
+        for (int x = 0; x < C::BOXES; ++x) {
+          tma_load_2d(sK + x * (kT * 128), &tmK, kv_full, item.h * DH + 64 * x, (int32_t)(s0 + k0));
+          tma_load_2d(sV + x * (kT * 128), &tmV, kv_full, item.h * DH + 64 * x, (int32_t)(s0 + k0));
+        }
+        kv_iss = true;
+        kv_par = items_done & 1;
+      }
+      ++items_done;
+      for (int qi = 0; qi < nqt; ++qi, ++m) {
+        const int q0 = (item.kt + qi) * kT;
+        if (lane == 0) ok = mbar_wait(qd_empty, (m & 1) ^ 1, abort_flag, P.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        long long* qts = reinterpret_cast<long long*>(sQD + C::QD_BYTES);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = lane + 32 * u;
+          qts[c] = (q0 + c < n) ? a.q_ts[s0 + q0 + c] : 0;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_expect_tx(qd_full, C::QD_BYTES);
+#pragma unroll
+          for (int x = 0; x < C::BOXES; ++x) {
+            tma_load_2d(sQD + x * (kT * 128), &tmQ, qd_full, item.h * DH + 64 * x, (int32_t)(s0 + q0));
+            tma_load_2d(sQD + C::TILE + x * (kT * 128), &tmdO, qd_full, item.h * DH + 64 * x,
+                        (int32_t)(s0 + q0));
+          }
+          qd_iss = true;
+          qd_par = m & 1;
+        }
+      }
+      if (!ok) break;
+    }
+    if (lane == 0) {
+      volatile int never = 0;
+      if (kv_iss) mbar_wait(kv_full, kv_par, &never, P.status);
+      if (qd_iss) mbar_wait(qd_full, qd_par, &never, P.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t items_done = 0, m = 0;
+      const uint32_t k_s = smem_u32(sK), v_s = smem_u32(sV), qd_s = smem_u32(sQD),
+                     ds_s = smem_u32(sDS);
+      for (int it = blockIdx.x; it < total; it += gridDim.x) {
+        if (*abort_flag) break;
+        const BItem item = P.w.items[it];
+        int64_t s0;
+        int n, hlen;
+        bgeom(a, item.b, s0, n, hlen);
+        const int nqt = bcost(n, item.kt);
+        if (!mbar_wait(kv_full, items_done & 1, abort_flag, P.status)) break;
+        if (!mbar_wait(dkv_free, (items_done & 1) ^ 1, abort_flag, P.status)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int qi = 0; qi < nqt; ++qi, ++m) {
+          if (!mbar_wait(qd_full, m & 1, abort_flag, P.status)) { ok = false; break; }
+          if (m > 0 && !mbar_wait(a_free, (m - 1) & 1, abort_flag, P.status)) { ok = false; break; }
+          tc_fence_after();
+          // S^T = K Q_i^T (region A), dP^T = V dO_i^T (region B)
+#pragma unroll
+          for (int k = 0; k < DH / 16; ++k) {
+            const uint32_t off = (k / 4) * (kT * 128) + (k % 4) * 32;
+            mma_ss(tA, sdesc_kmajor(k_s + off), sdesc_kmajor(qd_s + off), C::IDESC_ST, k > 0);
+          }
+#pragma unroll
+          for (int k = 0; k < DH / 16; ++k) {
+            const uint32_t off = (k / 4) * (kT * 128) + (k % 4) * 32;
+            mma_ss(tB, sdesc_kmajor(v_s + off), sdesc_kmajor(qd_s + C::TILE + off), C::IDESC_ST, k > 0);
+          }
+          mma_commit(st_full);
+          if (!mbar_wait(pds_full, m & 1, abort_flag, P.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t acc0 = qi > 0 ? 1u : 0u;
+          // dV += P^T dO_i ; dK += dS^T Q_i   (sum over the 128 queries)
+#pragma unroll
+          for (int k = 0; k < kT / 16; ++k)
+            mma_ts(tdV, tA + k * 8, sdesc_mnmajor(qd_s + C::TILE + k * 2048, kT * 128), C::IDESC_DKV,
+                   (acc0 || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < kT / 16; ++k)
+            mma_ts(tdK, tB + k * 8, sdesc_mnmajor(qd_s + k * 2048, kT * 128), C::IDESC_DKV,
+                   (acc0 || k > 0) ? 1u : 0u);
+          // dQ_i = dS K (sum over the 128 keys) into region A
+#pragma unroll
+          for (int k = 0; k < kT / 16; ++k)
+            mma_ss(tA, sdesc_mnmajor(ds_s + k * 2048, kT * 128), sdesc_mnmajor(k_s + k * 2048, kT * 128),
+                   C::IDESC_DQ, k > 0 ? 1u : 0u);
+          mma_commit(qd_empty);
+          mma_commit(dq_full);
+        }
+        if (!ok) break;
+        ++items_done;
+        mma_commit(kv_empty);
+        mma_commit(dkv_full);
+      }
+      mma_commit(done_bar);
+      volatile int never = 0;
+      mbar_wait(done_bar, 0, &never, P.status);
+    }
+  } else {
+    // ------------------------------------------------------------ key-row warps
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;             // key within the tile (TMEM lane)
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int d = P.A.d;
+    uint32_t items_done = 0, m = 0;
+    int cur_h = -1;
+    const float inv_N = a.inv_N;
+    for (int it = blockIdx.x; it < total; it += gridDim.x) {
+      const BItem item = P.w.items[it];
+      int64_t s0;
+      int n, hlen;
+      bgeom(a, item.b, s0, n, hlen);
+      const int k0 = item.kt * kT;
+      const int nqt = bcost(n, item.kt);
+      const int jk = k0 + row;                       // key index in the sequence
+      const bool kvalid = jk < hlen;
+      const long long tk = kvalid ? a.kv_ts[s0 + jk] : 0;
+      if (item.h != cur_h) {
+        named_barrier(1, 128);
+        if (cur_h >= 0 && row < 64) {
+          float* dst = row < 32 ? P.A.drab_pos : P.A.drab_time;
+          const int nb = row < 32 ? a.P : a.Bt;
+          const int bi = row & 31;
+          if (dst && bi < nb && drab[row] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[row]);
+        }
+        if (row < 32) {
+          rab[row] = (a.rab_pos && row < a.P) ? a.rab_pos[item.h * a.P + row] : 0.f;
+          rab[32 + row] = (a.rab_time && row < a.Bt) ? a.rab_time[item.h * a.Bt + row] : 0.f;
+        }
+        if (row < 64) drab[row] = 0.f;
+        named_barrier(1, 128);
+        cur_h = item.h;
+      }
+      bool fail = *abort_flag != 0;
+      if (named_barrier_any(1, 128, fail)) break;
+      for (int qi = 0; qi < nqt; ++qi, ++m) {
+        const int q0 = (item.kt + qi) * kT;
+        fail = !mbar_wait(st_full, m & 1, abort_flag, P.status);
+        if (named_barrier_any(1, 128, fail)) { fail = true; break; }
+        tc_fence_after();
+        const long long* qts = reinterpret_cast<const long long*>(sQD + C::QD_BYTES);
+        // run-length sums of dS per bucket along this key row (queries in
+        // increasing order: both buckets are monotone along the row)
+        int cur_bp = -1, cur_bt = -1;
+        float run_p = 0.f, run_t = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kT / 32; ++c) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tA + lane_off + c * 32, sr);
+          tmem_ld32(tB + lane_off + c * 32, dr);
+          tmem_ld_wait();
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int col = c * 32 + e + u;
+              const int qi_pos = q0 + col;           // query index in the sequence
+              const bool ok = kvalid && qi_pos < n && (qi_pos >= hlen || jk <= qi_pos);
+              float pa = 0.f, ds = 0.f;
+              if (ok) {
+                const int bp = min(max(min(qi_pos, hlen) - jk, 0), a.P - 1);
+                const long long dt = qts[col] - tk;
+                const int bt = dt <= 0 ? 0 : min(64 - __clzll(dt), a.Bt - 1);
+                const float x = __uint_as_float(sr[e + u]) + rab[bp] + rab[32 + bt];
+                const float sg = fmaf(0.5f, tanh_fast(0.5f * x), 0.5f);
+                pa = x * sg * inv_N;
+                ds = __uint_as_float(dr[e + u]) * sg * fmaf(x, 1.f - sg, 1.f) * inv_N;
+                if (bp != cur_bp) {
+                  if (cur_bp >= 0) atomicAdd(&drab[cur_bp], run_p);
+                  cur_bp = bp;
+                  run_p = 0.f;
+                }
+                run_p += ds;
+                if (bt != cur_bt) {
+                  if (cur_bt >= 0) atomicAdd(&drab[32 + cur_bt], run_t);
+                  cur_bt = bt;
+                  run_t = 0.f;
+                }
+                run_t += ds;
+              }
+              pv[u] = pa;
+              dv[u] = ds;
+            }
+            pk[e / 2] = pack_bf16(pv[0], pv[1]);
+            dk[e / 2] = pack_bf16(dv[0], dv[1]);
+          }
+          tmem_st16(tA + lane_off + c * 16, pk);
+          tmem_st16(tB + lane_off + c * 16, dk);
+          // dS[key][query] for the dQ MMA (queries are the MN dimension)
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) {
+            const uint4 v = make_uint4(dk[4 * g8], dk[4 * g8 + 1], dk[4 * g8 + 2], dk[4 * g8 + 3]);
+            *reinterpret_cast<uint4*>(sDS + mn_off(row, c * 32 + g8 * 8, kT * 128)) = v;
+          }
+        }
+        if (cur_bp >= 0) atomicAdd(&drab[cur_bp], run_p);
+        if (cur_bt >= 0) atomicAdd(&drab[32 + cur_bt], run_t);
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pds_full);
+        // drain dQ_i (TMEM lane = query row) into the fp32 accumulator
+        fail = !mbar_wait(dq_full, m & 1, abort_flag, P.status);
+        if (named_barrier_any(1, 128, fail)) { fail = true; break; }
+        tc_fence_after();
+        const int qrow = q0 + row;
+        float* dq = P.A.dq_acc + (s0 + qrow) * (int64_t)d + item.h * DH;
+#pragma unroll 1
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tA + lane_off + c * 32, r);
+          tmem_ld_wait();
+          if (qrow < n) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              red_add_v4(dq + c * 32 + i, __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                         __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(a_free);
+      }
+      if (fail) break;
+      // dK, dV of this key tile, times SiLU'(Pre), into dPre
+      fail = !mbar_wait(dkv_full, items_done & 1, abort_flag, P.status);
+      ++items_done;
+      if (named_barrier_any(1, 128, fail)) break;
+      tc_fence_after();
+      const bf16* pre = static_cast<const bf16*>(P.A.pre);
+      bf16* dpre = static_cast<bf16*>(P.A.dpre);
+      const int64_t rowoff = (s0 + jk) * P.A.pre_stride;
+#pragma unroll 1
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t rv[32], rk[32];
+        tmem_ld32(tdV + lane_off + c * 32, rv);
+        tmem_ld32(tdK + lane_off + c * 32, rk);
+        tmem_ld_wait();
+        if (kvalid) {
+          const int col = item.h * DH + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            const uint4 pv4 = *reinterpret_cast<const uint4*>(pre + rowoff + d + col + i);
+            const uint4 pk4 = *reinterpret_cast<const uint4*>(pre + rowoff + 3 * d + col + i);
+            const __nv_bfloat162* pvh = reinterpret_cast<const __nv_bfloat162*>(&pv4);
+            const __nv_bfloat162* pkh = reinterpret_cast<const __nv_bfloat162*>(&pk4);
+            uint4 ov, ok4;
+            uint32_t* ovw = reinterpret_cast<uint32_t*>(&ov);
+            uint32_t* okw = reinterpret_cast<uint32_t*>(&ok4);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 fv = __bfloat1622float2(pvh[u]);
+              const float2 fk = __bfloat1622float2(pkh[u]);
+              ovw[u] = pack_bf16(__uint_as_float(rv[i + 2 * u]) * silu_grad_acc(fv.x),
+                                 __uint_as_float(rv[i + 2 * u + 1]) * silu_grad_acc(fv.y));
+              okw[u] = pack_bf16(__uint_as_float(rk[i + 2 * u]) * silu_grad_acc(fk.x),
+                                 __uint_as_float(rk[i + 2 * u + 1]) * silu_grad_acc(fk.y));
+            }
+            *reinterpret_cast<uint4*>(dpre + rowoff + d + col + i) = ov;
+            *reinterpret_cast<uint4*>(dpre + rowoff + 3 * d + col + i) = ok4;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dkv_free);
+    }
+    // flush the last head's bucket sums
+    named_barrier(1, 128);
+    if (cur_h >= 0 && row < 64) {
+      float* dst = row < 32 ? P.A.drab_pos : P.A.drab_time;
+      const int nb = row < 32 ? a.P : a.Bt;
+      const int bi = row & 31;
+      if (dst && bi < nb && drab[row] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[row]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+int sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int DH>
+cudaError_t launch_bwd(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaStream_t s) {
+  using C = BCfg<DH>;
+  const AttnArgs& a = A.f;
+  const int d = a.H * DH;
+  CUtensorMap tQ, tK, tV, tdO;
+  bool ok = encode_tmap_2d(&tQ, false, a.q, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)a.q_stride, 64, kT) &&
+            encode_tmap_2d(&tK, false, a.k, (uint64_t)d, (uint64_t)a.kv_rows, (uint64_t)a.kv_stride, 64, kT) &&
+            encode_tmap_2d(&tV, false, a.v, (uint64_t)d, (uint64_t)a.kv_rows, (uint64_t)a.kv_stride, 64, kT) &&
+            encode_tmap_2d(&tdO, false, A.dout, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)a.o_stride, 64, kT);
+  if (!ok) return cudaErrorInvalidValue;
+  BSched w = bsched(ws);
+  cudaError_t e = cudaMemsetAsync(w.hist, 0, 3 * kMaxCostB * sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
+  const int blocks = (a.B + 255) / 256;
+  bsched_count<<<blocks, 256, 0, s>>>(a, w);
+  bsched_scan<<<1, 32, 0, s>>>(w);
+  bsched_fill<<<blocks, 256, 0, s>>>(a, w);
+  count_launch(3);
+  BParams P;
+  P.A = A;
+  P.w = w;
+  P.status = status;
+  auto kern = attn_bwd_tc_kernel<DH>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<sms(), 192, C::SMEM, s>>>(tQ, tK, tV, tdO, P);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attn_bwd_sched_bytes(int B, int64_t T, int H) {
+  const size_t max_items = ((size_t)(T / kT) + (size_t)B + 1) * (size_t)H;
+  return align_up(3 * kMaxCostB * sizeof(int32_t), 256) + max_items * sizeof(BItem);
+}
+
+bool attention_bwd_tc_supported(int dtype, const AttnBwdArgs& A) {
+  const AttnArgs& a = A.f;
+  return dtype == HSTU_BF16 && (a.dh == 64 || a.dh == 128) && !a.cached && a.q_rows > 0 &&
+         a.q_stride % 8 == 0 && a.kv_stride % 8 == 0 && a.o_stride % 8 == 0 && a.P <= 32 &&
+         a.Bt <= 32;
+}
+
+cudaError_t attention_bwd_tc(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaStream_t s) {
+  if (A.f.dh == 128) return launch_bwd<128>(A, ws, status, s);
+  return launch_bwd<64>(A, ws, status, s);
+}
+
+}  // namespace hstu

@@ -487,7 +487,26 @@ cudaError_t bwd_dh(const AttnBwdArgs& a, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
+template <typename T>
+cudaError_t self_dh(const AttnBwdArgs& a, cudaStream_t s) {
+  dim3 g2(4, (unsigned)a.f.B, (unsigned)a.f.H);
+  switch (a.f.dh) {
+    case 32: attn_bwd_self_kernel<T, 32><<<g2, 256, 0, s>>>(a); break;
+    case 64: attn_bwd_self_kernel<T, 64><<<g2, 256, 0, s>>>(a); break;
+    case 128: attn_bwd_self_kernel<T, 128><<<g2, 256, 0, s>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  count_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+// Candidate keys' dK, dV and their dQ contribution (the self term).
+cudaError_t attention_bwd_self_simt(int dtype, const AttnBwdArgs& a, cudaStream_t s) {
+  if (!a.f.num_targets || a.f.B == 0) return cudaSuccess;
+  return dtype == HSTU_BF16 ? self_dh<bf16>(a, s) : self_dh<float>(a, s);
+}
 
 cudaError_t attention_fwd_simt(int dtype, const AttnArgs& a, cudaStream_t s) {
   return dtype == HSTU_BF16 ? fwd_dh<bf16>(a, s) : fwd_dh<float>(a, s);

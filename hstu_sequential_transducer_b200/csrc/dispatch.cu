@@ -22,8 +22,12 @@ cudaError_t attention_fwd(int dtype, const AttnArgs& a, void* ws, size_t ws_byte
 
 cudaError_t attention_bwd(int dtype, const AttnBwdArgs& a, void* ws, size_t ws_bytes,
                           cudaStream_t s) {
-  (void)ws;
-  (void)ws_bytes;
+  if (attention_bwd_tc_supported(dtype, a) &&
+      ws_bytes >= attn_bwd_sched_bytes(a.f.B, a.f.q_rows, a.f.H)) {
+    cudaError_t e = attention_bwd_tc(a, ws, device_status(), s);
+    if (e != cudaSuccess) return e;
+    return attention_bwd_self_simt(dtype, a, s);
+  }
   return attention_bwd_simt(dtype, a, s);
 }
 
@@ -32,8 +36,9 @@ size_t attention_fwd_ws(int B, int64_t T, int H, int max_len) {
   return attn_sched_bytes(B, T, H);
 }
 size_t attention_bwd_ws(int B, int64_t T, int H, int d, int max_len) {
-  (void)B; (void)T; (void)H; (void)d; (void)max_len;
-  return 0;
+  (void)d;
+  (void)max_len;
+  return attn_bwd_sched_bytes(B, T, H);
 }
 
 }  // namespace hstu

@@ -95,6 +95,10 @@ size_t attn_sched_bytes(int B, int64_t Tq, int H);
 bool attention_fwd_tc_supported(int dtype, const AttnArgs& a);
 cudaError_t attention_fwd_tc(const AttnArgs& a, void* ws, uint32_t* status, cudaStream_t s);
 size_t attention_bwd_ws(int B, int64_t T, int H, int d, int max_len);
+size_t attn_bwd_sched_bytes(int B, int64_t T, int H);
+bool attention_bwd_tc_supported(int dtype, const AttnBwdArgs& a);
+cudaError_t attention_bwd_tc(const AttnBwdArgs& a, void* ws, uint32_t* status, cudaStream_t s);
+cudaError_t attention_bwd_self_simt(int dtype, const AttnBwdArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // LayerNorm (.) U epilogue

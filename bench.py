@@ -72,10 +72,16 @@ def describe(w: W.Workload):
     }[w.name.replace("_subset", "")]
 
 
-def make_workload(name, rank):
+def make_workload(name, rank, batch=None):
+    """The named workload; `batch` keeps only its first sequences (a small
+    case of the same shapes, e.g. for profiler captures)."""
     if name == "training":
-        return W.training(data_seed=5 + 1000 * rank)
-    return W.WORKLOADS[name]()
+        w = W.training(data_seed=5 + 1000 * rank)
+    else:
+        w = W.WORKLOADS[name]()
+    if batch is not None and batch < w.B:
+        w = W.subset(w, list(range(batch)))
+    return w
 
 
 # ----------------------------------------------------------------------------
@@ -188,7 +194,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = make_workload(args.workload, 0)
+    w = make_workload(args.workload, 0, args.batch)
     for _ in range(args.warmup):
         oracle_sample(w, 0.0)
     vals, times = [], []
@@ -237,13 +243,13 @@ def run_ours(args):
         dist.barrier()
     H.lib()
 
-    w = make_workload(args.workload, rank)
+    w = make_workload(args.workload, rank, args.batch)
     dw = S.DeviceWorkload.from_workload(w)
     backward = w.backward
     flops, pairs = workload_flops(w, backward)
     dev = torch.device("cuda", local)
 
-    if args.workload == "mfalcon":
+    if args.workload == "mfalcon" and args.batch is None:
         hist, cand = w.meta["history"], w.meta["candidates"]
 
         def step():
@@ -337,7 +343,7 @@ def run_ours(args):
 
     # end to end through the public API with host buffers
     e2e = None
-    if backward and args.workload == "training" and not args.skip_e2e:
+    if backward and args.workload == "training" and not args.skip_e2e and args.batch is None:
         e2e = e2e_training(args, ts, dw, world, dist)
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -416,6 +422,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="keep only the first B sequences (a small case for profiler captures)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)

@@ -16,12 +16,22 @@
 //   warp 1      MMA issuer: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM; then
 //               dV += P^T dO_i and dK += dS^T Q_i (P^T, dS^T as TMEM A
 //               operands) and dQ_i = dS K (dS from shared memory)
-//   warps 2..5  one key row per thread: P^T and dS^T from S^T, dP^T; dS into
-//               shared memory; run-length sums of dS per rab bucket; then dQ_i
-//               from TMEM into the fp32 dQ accumulator (vector reductions);
-//               after the last query tile dK, dV times SiLU'(Pre) to dPre
+//   warps 2..9  two warpgroups, one key row per thread, each taking half of the
+//               128 query columns: P^T and dS^T from S^T, dP^T (unscaled by
+//               1/N, which the drains apply); dS into shared memory; sums of
+//               dS per rab bucket; then their half of dQ_i from TMEM into the
+//               fp32 dQ accumulator (vector reductions); after the last query
+//               tile their half of dK, dV times SiLU'(Pre) to dPre
 // TMEM (512 columns): [0,128) S^T -> P^T -> dQ_i, [128,256) dP^T -> dS^T,
-// [256,384) dV, [384,512) dK.
+// [256,384) dV, [384,512) dK.  Each warpgroup writes its P^T (dS^T) into the
+// first half of its own S^T (dP^T) columns, so the two never overwrite
+// values the other still reads; the dV and dK MMAs address the two
+// 64-query halves of the A operand separately.
+//
+// As in the forward, away from the diagonal the rab bias of a key row
+// against a query tile is a step function with at most two breakpoints along
+// the row (time buckets are non-decreasing in the query's time), and so are
+// the per-bucket sums of dS: a total and one suffix sum per breakpoint.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -127,17 +137,66 @@ struct BParams {
   uint32_t* status;
 };
 
+__device__ __forceinline__ float tanh_fast(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
+  return t;
+}
+
+constexpr int kBThreads = 320;
+constexpr int kActWarps = 8;
+
+__device__ __forceinline__ int tb64(long long dt, int Bt) {
+  return dt <= 0 ? 0 : min(64 - __clzll(dt), Bt - 1);
+}
+
+// Number of the 128 non-decreasing values cts[] that are <= tau.
+__device__ __forceinline__ int count_le_128(const long long* cts, long long tau) {
+  if (cts[127] <= tau) return 128;
+  int lo = 0;
+#pragma unroll
+  for (int step = 64; step >= 1; step >>= 1)
+    if (cts[lo + step - 1] <= tau) lo += step;
+  return lo;
+}
+
+// One 32-column chunk of the fast path: h = S/2 + bias/2 where columns
+// c >= p[k] add hd[k]; writes packed P and dS (unscaled) and accumulates the
+// total and the per-breakpoint suffix sums of dS.
+template <int NB>
+__device__ __forceinline__ void bwd_chunk_fast(const uint32_t (&sr)[32], const uint32_t (&dr)[32],
+                                               int c0, float hb, const int (&p)[2],
+                                               const float (&hd)[2], uint32_t (&pk)[16],
+                                               uint32_t (&dk)[16], float& tot, float (&suf)[2]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float pa[2], ds[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = c0 + e + u;
+      float h = fmaf(__uint_as_float(sr[e + u]), 0.5f, hb);
+#pragma unroll
+      for (int k = 0; k < NB; ++k) h += (c >= p[k]) ? hd[k] : 0.f;
+      const float t = tanh_fast(h);
+      const float sg = fmaf(t, 0.5f, 0.5f);
+      pa[u] = fmaf(h, t, h);                       // SiLU(x)
+      const float w = fmaf(-h, t, h);              // x (1 - sigmoid(x))
+      ds[u] = __uint_as_float(dr[e + u]) * fmaf(sg, w, sg);
+      tot += ds[u];
+#pragma unroll
+      for (int k = 0; k < NB; ++k) suf[k] += (c >= p[k]) ? ds[u] : 0.f;
+    }
+    pk[e / 2] = pack_bf16(pa[0], pa[1]);
+    dk[e / 2] = pack_bf16(ds[0], ds[1]);
+  }
+}
+
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
                "f"(d)
                : "memory");
 }
 
-__device__ __forceinline__ float tanh_fast(float x) {
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(x));
-  return t;
-}
 
 // Byte offset of (row k, column c) in a 128-byte-swizzled MN-major tile whose
 // MN extent (c) is split into 64-wide blocks `blk` bytes apart and whose K
@@ -148,7 +207,7 @@ __device__ __forceinline__ uint32_t mn_off(int k, int c, uint32_t blk) {
 }
 
 template <int DH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kBThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                        const BParams P) {
@@ -182,8 +241,8 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 11; ++i) {
-      const bool four = &bars[i] == pds_full || &bars[i] == a_free || &bars[i] == dkv_free;
-      mbar_init(&bars[i], four ? 4 : 1);
+      const bool act = &bars[i] == pds_full || &bars[i] == a_free || &bars[i] == dkv_free;
+      mbar_init(&bars[i], act ? kActWarps : 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -232,7 +291,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int c = lane + 32 * u;
-          qts[c] = (q0 + c < n) ? a.q_ts[s0 + q0 + c] : 0;
+          // past the sequence: a large sentinel keeps the staged times sorted
+          qts[c] = (q0 + c < n) ? a.q_ts[s0 + q0 + c] : (1LL << 62);
         }
         __syncwarp();
         if (lane == 0) {
@@ -291,14 +351,15 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after();
           const uint32_t acc0 = qi > 0 ? 1u : 0u;
           // dV += P^T dO_i ; dK += dS^T Q_i   (sum over the 128 queries)
+          // A operand halves: queries [0,64) at columns [0,32), [64,128) at [64,96)
 #pragma unroll
           for (int k = 0; k < kT / 16; ++k)
-            mma_ts(tdV, tA + k * 8, sdesc_mnmajor(qd_s + C::TILE + k * 2048, kT * 128), C::IDESC_DKV,
-                   (acc0 || k > 0) ? 1u : 0u);
+            mma_ts(tdV, tA + (k / 4) * 64 + (k % 4) * 8, sdesc_mnmajor(qd_s + C::TILE + k * 2048, kT * 128),
+                   C::IDESC_DKV, (acc0 || k > 0) ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < kT / 16; ++k)
-            mma_ts(tdK, tB + k * 8, sdesc_mnmajor(qd_s + k * 2048, kT * 128), C::IDESC_DKV,
-                   (acc0 || k > 0) ? 1u : 0u);
+            mma_ts(tdK, tB + (k / 4) * 64 + (k % 4) * 8, sdesc_mnmajor(qd_s + k * 2048, kT * 128),
+                   C::IDESC_DKV, (acc0 || k > 0) ? 1u : 0u);
           // dQ_i = dS K (sum over the 128 keys) into region A
 #pragma unroll
           for (int k = 0; k < kT / 16; ++k)
@@ -319,12 +380,15 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ------------------------------------------------------------ key-row warps
     const int quarter = warp & 3;
+    const int wg = (warp - 2) >> 2;                  // query columns [64 wg, 64 wg + 64)
     const int row = quarter * 32 + lane;             // key within the tile (TMEM lane)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    constexpr uint32_t kAct = 32 * kActWarps;
     const int d = P.A.d;
     uint32_t items_done = 0, m = 0;
     int cur_h = -1;
     const float inv_N = a.inv_N;
+    const int ti = threadIdx.x - 64;                 // 0..255
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
       const BItem item = P.w.items[it];
       int64_t s0;
@@ -336,108 +400,164 @@ __global__ void __launch_bounds__(192, 1)
       const bool kvalid = jk < hlen;
       const long long tk = kvalid ? a.kv_ts[s0 + jk] : 0;
       if (item.h != cur_h) {
-        named_barrier(1, 128);
-        if (cur_h >= 0 && row < 64) {
-          float* dst = row < 32 ? P.A.drab_pos : P.A.drab_time;
-          const int nb = row < 32 ? a.P : a.Bt;
-          const int bi = row & 31;
-          if (dst && bi < nb && drab[row] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[row]);
+        named_barrier(1, kAct);
+        if (cur_h >= 0 && ti < 64) {
+          float* dst = ti < 32 ? P.A.drab_pos : P.A.drab_time;
+          const int nb = ti < 32 ? a.P : a.Bt;
+          const int bi = ti & 31;
+          if (dst && bi < nb && drab[ti] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[ti] * inv_N);
         }
-        if (row < 32) {
-          rab[row] = (a.rab_pos && row < a.P) ? a.rab_pos[item.h * a.P + row] : 0.f;
-          rab[32 + row] = (a.rab_time && row < a.Bt) ? a.rab_time[item.h * a.Bt + row] : 0.f;
+        if (ti < 32) {
+          rab[ti] = (a.rab_pos && ti < a.P) ? a.rab_pos[item.h * a.P + ti] : 0.f;
+          rab[32 + ti] = (a.rab_time && ti < a.Bt) ? a.rab_time[item.h * a.Bt + ti] : 0.f;
         }
-        if (row < 64) drab[row] = 0.f;
-        named_barrier(1, 128);
+        if (ti < 64) drab[ti] = 0.f;
+        named_barrier(1, kAct);
         cur_h = item.h;
       }
       bool fail = *abort_flag != 0;
-      if (named_barrier_any(1, 128, fail)) break;
+      if (named_barrier_any(1, kAct, fail)) break;
+      const float rp_far = rab[a.P - 1];
       for (int qi = 0; qi < nqt; ++qi, ++m) {
         const int q0 = (item.kt + qi) * kT;
         fail = !mbar_wait(st_full, m & 1, abort_flag, P.status);
-        if (named_barrier_any(1, 128, fail)) { fail = true; break; }
+        if (named_barrier_any(1, kAct, fail)) { fail = true; break; }
         tc_fence_after();
         const long long* qts = reinterpret_cast<const long long*>(sQD + C::QD_BYTES);
-        // run-length sums of dS per bucket along this key row (queries in
-        // increasing order: both buckets are monotone along the row)
-        int cur_bp = -1, cur_bt = -1;
-        float run_p = 0.f, run_t = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < kT / 32; ++c) {
-          uint32_t sr[32], dr[32];
-          tmem_ld32(tA + lane_off + c * 32, sr);
-          tmem_ld32(tB + lane_off + c * 32, dr);
-          tmem_ld_wait();
-          uint32_t pk[16], dk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pv[2], dv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int col = c * 32 + e + u;
-              const int qi_pos = q0 + col;           // query index in the sequence
-              const bool ok = kvalid && qi_pos < n && (qi_pos >= hlen || jk <= qi_pos);
-              float pa = 0.f, ds = 0.f;
-              if (ok) {
-                const int bp = min(max(min(qi_pos, hlen) - jk, 0), a.P - 1);
-                const long long dt = qts[col] - tk;
-                const int bt = dt <= 0 ? 0 : min(64 - __clzll(dt), a.Bt - 1);
-                const float x = __uint_as_float(sr[e + u]) + rab[bp] + rab[32 + bt];
-                const float sg = fmaf(0.5f, tanh_fast(0.5f * x), 0.5f);
-                pa = x * sg * inv_N;
-                ds = __uint_as_float(dr[e + u]) * sg * fmaf(x, 1.f - sg, 1.f) * inv_N;
-                if (bp != cur_bp) {
-                  if (cur_bp >= 0) atomicAdd(&drab[cur_bp], run_p);
-                  cur_bp = bp;
-                  run_p = 0.f;
-                }
-                run_p += ds;
-                if (bt != cur_bt) {
-                  if (cur_bt >= 0) atomicAdd(&drab[32 + cur_bt], run_t);
-                  cur_bt = bt;
-                  run_t = 0.f;
-                }
-                run_t += ds;
-              }
-              pv[u] = pa;
-              dv[u] = ds;
-            }
-            pk[e / 2] = pack_bf16(pv[0], pv[1]);
-            dk[e / 2] = pack_bf16(dv[0], dv[1]);
-          }
-          tmem_st16(tA + lane_off + c * 16, pk);
-          tmem_st16(tB + lane_off + c * 16, dk);
-          // dS[key][query] for the dQ MMA (queries are the MN dimension)
-#pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8) {
-            const uint4 v = make_uint4(dk[4 * g8], dk[4 * g8 + 1], dk[4 * g8 + 2], dk[4 * g8 + 3]);
-            *reinterpret_cast<uint4*>(sDS + mn_off(row, c * 32 + g8 * 8, kT * 128)) = v;
-          }
+        const int qf = q0 + wg * 64;                 // first query of this warpgroup's half
+        // fast path: all 64 queries valid and causally after the key, last
+        // position bucket, at most two time-bucket breakpoints
+        const bool full = kvalid && qf + 63 < n && jk <= qf;
+        const bool far = min(qf, hlen) - jk >= a.P - 1;
+        int nb = 3, b_lo = 0;
+        if (full && far) {
+          b_lo = tb64(qts[wg * 64] - tk, a.Bt);
+          const int b_hi = tb64(qts[wg * 64 + 63] - tk, a.Bt);
+          nb = b_hi - b_lo;
         }
-        if (cur_bp >= 0) atomicAdd(&drab[cur_bp], run_p);
-        if (cur_bt >= 0) atomicAdd(&drab[32 + cur_bt], run_t);
+        const bool fast = __all_sync(0xffffffffu, full && far && nb <= 2);
+        const uint32_t sA = tA + lane_off + wg * 64, sB = tB + lane_off + wg * 64;
+        if (fast) {
+          const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)nb);
+          int p[2] = {64, 64};
+          float hd[2] = {0.f, 0.f};
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+            if (k < nb) {
+              const int b = b_lo + 1 + k;
+              // queries with t_q - t_k >= 2^(b-1): columns c >= p
+              p[k] = count_le_128(qts, tk + (1LL << (b - 1)) - 1) - wg * 64;
+              hd[k] = 0.5f * (rab[32 + b] - rab[32 + b - 1]);
+            }
+          const float hb = 0.5f * (rp_far + rab[32 + b_lo]);
+          float tot = 0.f, suf[2] = {0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t sr[32], dr[32], pk[16], dk[16];
+            tmem_ld32(sA + c * 32, sr);
+            tmem_ld32(sB + c * 32, dr);
+            tmem_ld_wait();
+            if (nbw == 0) bwd_chunk_fast<0>(sr, dr, c * 32, hb, p, hd, pk, dk, tot, suf);
+            else if (nbw == 1) bwd_chunk_fast<1>(sr, dr, c * 32, hb, p, hd, pk, dk, tot, suf);
+            else bwd_chunk_fast<2>(sr, dr, c * 32, hb, p, hd, pk, dk, tot, suf);
+            tmem_st16(sA + c * 16, pk);
+            tmem_st16(sB + c * 16, dk);
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+              const uint4 v = make_uint4(dk[4 * g8], dk[4 * g8 + 1], dk[4 * g8 + 2], dk[4 * g8 + 3]);
+              *reinterpret_cast<uint4*>(sDS + mn_off(row, wg * 64 + c * 32 + g8 * 8, kT * 128)) = v;
+            }
+          }
+          // bucket sums: b_lo + k + 1 gets suf[k] - suf[k+1], b_lo gets tot - suf[0]
+          if (kvalid) {
+            atomicAdd(&drab[a.P - 1], tot);
+            float below = tot;
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+              if (k < nb) {
+                atomicAdd(&drab[32 + b_lo + k], below - suf[k]);
+                below = suf[k];
+              }
+            atomicAdd(&drab[32 + b_lo + nb], below);
+          }
+        } else {
+          int cur_bp = -1, cur_bt = -1;
+          float run_p = 0.f, run_t = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t sr[32], dr[32], pk[16], dk[16];
+            tmem_ld32(sA + c * 32, sr);
+            tmem_ld32(sB + c * 32, dr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float pv[2], dv[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int col = wg * 64 + c * 32 + e + u;
+                const int qpos = q0 + col;
+                const bool ok = kvalid && qpos < n && (qpos >= hlen || jk <= qpos);
+                float pa = 0.f, ds = 0.f;
+                if (ok) {
+                  const int bp = min(max(min(qpos, hlen) - jk, 0), a.P - 1);
+                  const int bt = tb64(qts[col] - tk, a.Bt);
+                  const float h = 0.5f * (__uint_as_float(sr[e + u]) + rab[bp] + rab[32 + bt]);
+                  const float t = tanh_fast(h);
+                  const float sg = fmaf(t, 0.5f, 0.5f);
+                  pa = fmaf(h, t, h);
+                  ds = __uint_as_float(dr[e + u]) * fmaf(sg, fmaf(-h, t, h), sg);
+                  if (bp != cur_bp) {
+                    if (cur_bp >= 0) atomicAdd(&drab[cur_bp], run_p);
+                    cur_bp = bp;
+                    run_p = 0.f;
+                  }
+                  run_p += ds;
+                  if (bt != cur_bt) {
+                    if (cur_bt >= 0) atomicAdd(&drab[32 + cur_bt], run_t);
+                    cur_bt = bt;
+                    run_t = 0.f;
+                  }
+                  run_t += ds;
+                }
+                pv[u] = pa;
+                dv[u] = ds;
+              }
+              pk[e / 2] = pack_bf16(pv[0], pv[1]);
+              dk[e / 2] = pack_bf16(dv[0], dv[1]);
+            }
+            tmem_st16(sA + c * 16, pk);
+            tmem_st16(sB + c * 16, dk);
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+              const uint4 v = make_uint4(dk[4 * g8], dk[4 * g8 + 1], dk[4 * g8 + 2], dk[4 * g8 + 3]);
+              *reinterpret_cast<uint4*>(sDS + mn_off(row, wg * 64 + c * 32 + g8 * 8, kT * 128)) = v;
+            }
+          }
+          if (cur_bp >= 0) atomicAdd(&drab[cur_bp], run_p);
+          if (cur_bt >= 0) atomicAdd(&drab[32 + cur_bt], run_t);
+        }
         tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(pds_full);
-        // drain dQ_i (TMEM lane = query row) into the fp32 accumulator
+        // drain this warpgroup's half of dQ_i (TMEM lane = query row)
         fail = !mbar_wait(dq_full, m & 1, abort_flag, P.status);
-        if (named_barrier_any(1, 128, fail)) { fail = true; break; }
+        if (named_barrier_any(1, kAct, fail)) { fail = true; break; }
         tc_fence_after();
         const int qrow = q0 + row;
         float* dq = P.A.dq_acc + (s0 + qrow) * (int64_t)d + item.h * DH;
 #pragma unroll 1
-        for (int c = 0; c < DH / 32; ++c) {
+        for (int cc = 0; cc < DH / 64; ++cc) {
+          const int c = wg * (DH / 64) + cc;
           uint32_t r[32];
           tmem_ld32(tA + lane_off + c * 32, r);
           tmem_ld_wait();
           if (qrow < n) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
-              red_add_v4(dq + c * 32 + i, __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                         __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+              red_add_v4(dq + c * 32 + i, __uint_as_float(r[i]) * inv_N, __uint_as_float(r[i + 1]) * inv_N,
+                         __uint_as_float(r[i + 2]) * inv_N, __uint_as_float(r[i + 3]) * inv_N);
           }
         }
         tc_fence_before();
@@ -445,16 +565,17 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) mbar_arrive(a_free);
       }
       if (fail) break;
-      // dK, dV of this key tile, times SiLU'(Pre), into dPre
+      // this warpgroup's half of dK, dV (times 1/N and SiLU'(Pre)) into dPre
       fail = !mbar_wait(dkv_full, items_done & 1, abort_flag, P.status);
       ++items_done;
-      if (named_barrier_any(1, 128, fail)) break;
+      if (named_barrier_any(1, kAct, fail)) break;
       tc_fence_after();
       const bf16* pre = static_cast<const bf16*>(P.A.pre);
       bf16* dpre = static_cast<bf16*>(P.A.dpre);
       const int64_t rowoff = (s0 + jk) * P.A.pre_stride;
 #pragma unroll 1
-      for (int c = 0; c < DH / 32; ++c) {
+      for (int cc = 0; cc < DH / 64; ++cc) {
+        const int c = wg * (DH / 64) + cc;
         uint32_t rv[32], rk[32];
         tmem_ld32(tdV + lane_off + c * 32, rv);
         tmem_ld32(tdK + lane_off + c * 32, rk);
@@ -474,10 +595,10 @@ __global__ void __launch_bounds__(192, 1)
             for (int u = 0; u < 4; ++u) {
               const float2 fv = __bfloat1622float2(pvh[u]);
               const float2 fk = __bfloat1622float2(pkh[u]);
-              ovw[u] = pack_bf16(__uint_as_float(rv[i + 2 * u]) * silu_grad_acc(fv.x),
-                                 __uint_as_float(rv[i + 2 * u + 1]) * silu_grad_acc(fv.y));
-              okw[u] = pack_bf16(__uint_as_float(rk[i + 2 * u]) * silu_grad_acc(fk.x),
-                                 __uint_as_float(rk[i + 2 * u + 1]) * silu_grad_acc(fk.y));
+              ovw[u] = pack_bf16(__uint_as_float(rv[i + 2 * u]) * inv_N * silu_grad_acc(fv.x),
+                                 __uint_as_float(rv[i + 2 * u + 1]) * inv_N * silu_grad_acc(fv.y));
+              okw[u] = pack_bf16(__uint_as_float(rk[i + 2 * u]) * inv_N * silu_grad_acc(fk.x),
+                                 __uint_as_float(rk[i + 2 * u + 1]) * inv_N * silu_grad_acc(fk.y));
             }
             *reinterpret_cast<uint4*>(dpre + rowoff + d + col + i) = ov;
             *reinterpret_cast<uint4*>(dpre + rowoff + 3 * d + col + i) = ok4;
@@ -489,12 +610,12 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) mbar_arrive(dkv_free);
     }
     // flush the last head's bucket sums
-    named_barrier(1, 128);
-    if (cur_h >= 0 && row < 64) {
-      float* dst = row < 32 ? P.A.drab_pos : P.A.drab_time;
-      const int nb = row < 32 ? a.P : a.Bt;
-      const int bi = row & 31;
-      if (dst && bi < nb && drab[row] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[row]);
+    named_barrier(1, kAct);
+    if (cur_h >= 0 && ti < 64) {
+      float* dst = ti < 32 ? P.A.drab_pos : P.A.drab_time;
+      const int nb = ti < 32 ? a.P : a.Bt;
+      const int bi = ti & 31;
+      if (dst && bi < nb && drab[ti] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[ti] * inv_N);
     }
   }
 
@@ -543,7 +664,7 @@ cudaError_t launch_bwd(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaStr
   auto kern = attn_bwd_tc_kernel<DH>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<sms(), 192, C::SMEM, s>>>(tQ, tK, tV, tdO, P);
+  kern<<<sms(), kBThreads, C::SMEM, s>>>(tQ, tK, tV, tdO, P);
   count_launch();
   return cudaGetLastError();
 }

@@ -14,11 +14,21 @@
 //               the keys' timestamps into a ring of stages
 //   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S
 //               buffers; O += P V with P read from TMEM (A operand in TMEM)
-//   warps 2..5  one query row per thread: S from TMEM, bucketed rab bias, mask,
-//               SiLU, P (bf16) written back over S; at the end of an item, O
-//               from TMEM times 1/N plus the candidates' self term, to HBM
-// tcgen05.mma instructions of one thread execute in issue order, so the QK^T
-// of tile j+2 overwrites S/P buffer j%2 only after the PV of tile j read it.
+//   warps 2..9  two warpgroups, one query row per thread, each taking half of
+//               the 128 key columns: S from TMEM, bucketed rab bias, mask,
+//               SiLU, P (bf16) into a TMEM P buffer; at the end of an item,
+//               half of O each, times 1/N plus the candidates' self term
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O [256,384), P0 [384,448),
+// P1 [448,512).  A commit arrives only when every earlier MMA of the thread
+// is complete, so once S_{j+2} is signalled the PV of tile j has read P_j.
+//
+// The rab bias of one row against one key tile is cheap in the common case:
+// away from the diagonal the position bucket is the last one, and the time
+// bucket, a non-increasing step function of the key (timestamps are
+// non-decreasing), changes at no more than two breakpoints, found by binary
+// search over the tile's timestamps once per row and tile.  Rows of a warp
+// that all qualify take that path (a few compares per element); the others
+// (diagonal, tails, candidates' near keys) evaluate buckets per element.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -162,7 +172,9 @@ struct FwdCfg {
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr uint32_t IDESC_S = idesc_bf16(128, kTile, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16(128, DH, false, true);
-  static constexpr uint32_t TMEM_COLS = 512;            // S0, S1, O
+  static constexpr uint32_t TMEM_COLS = 512;            // S0, S1, O, P0, P1
+  static constexpr int THREADS = 320;
+  static constexpr int ACT_WARPS = 8;
 };
 
 struct FwdParams {
@@ -171,16 +183,51 @@ struct FwdParams {
   uint32_t* status;
 };
 
-__device__ __forceinline__ float silu_fast(float x) {
-  // x * sigmoid(x) = h + h * tanh(h) with h = x / 2
-  const float h = 0.5f * x;
+// SiLU(x) from h = x / 2:  x * sigmoid(x) = h + h * tanh(h)
+__device__ __forceinline__ float silu_half(float h) {
   float t;
   asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
   return fmaf(h, t, h);
 }
 
+__device__ __forceinline__ int time_bucket32(long long dt, int Bt) {
+  return dt <= 0 ? 0 : min(64 - __clzll(dt), Bt - 1);
+}
+
+// Number of the 128 non-decreasing values cts[] that are <= tau.
+__device__ __forceinline__ int count_le128(const long long* cts, long long tau) {
+  if (cts[127] <= tau) return 128;
+  int lo = 0;
+#pragma unroll
+  for (int step = 64; step >= 1; step >>= 1)
+    if (cts[lo + step - 1] <= tau) lo += step;
+  return lo;
+}
+
+// Activation of one 32-column chunk in the fast path: h = S/2 + bias/2 with
+// the bias a step function (NB breakpoints, columns c < p[k] add hd[k]);
+// returns packed bf16 SiLU values.
+template <int NB>
+__device__ __forceinline__ void act_chunk_fast(const uint32_t (&s)[32], int c0, float hb,
+                                               const int (&p)[2], const float (&hd)[2],
+                                               uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float y[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = c0 + e + u;
+      float h = fmaf(__uint_as_float(s[e + u]), 0.5f, hb);
+#pragma unroll
+      for (int k = 0; k < NB; ++k) h += (c < p[k]) ? hd[k] : 0.f;
+      y[u] = silu_half(h);
+    }
+    pk[e / 2] = pack_bf16(y[0], y[1]);
+  }
+}
+
 template <int DH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const FwdParams P) {
   using C = FwdCfg<DH>;
@@ -215,10 +262,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], C::ACT_WARPS);
     }
     mbar_init(o_full, 1);
-    mbar_init(o_free, 4);
+    mbar_init(o_free, C::ACT_WARPS);
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -230,6 +277,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS[2] = {tmem, tmem + 128};
   const uint32_t tO = tmem + 256;
+  const uint32_t tP[2] = {tmem + 384, tmem + 448};
 
   // Every role walks the same item sequence and numbers the key tiles it
   // meets with one running counter n: K/V stage n % STAGES (parity
@@ -273,7 +321,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int c = lane + 32 * q;
-          kts[c] = (k0 + c < kend) ? a.kv_ts[g.ks + k0 + c] : 0;
+          // past the visible keys: a large sentinel keeps the staged times sorted
+          kts[c] = (k0 + c < kend) ? a.kv_ts[g.ks + k0 + c] : (1LL << 62);
         }
         __syncwarp();
         if (lane == 0) {
@@ -309,7 +358,6 @@ __global__ void __launch_bounds__(192, 1)
         const int nk = (kend + kTile - 1) / kTile;
         if (nk == 0) continue;
         if (!mbar_wait(q_full, items_done & 1, abort_flag, P.status)) break;
-        if (!mbar_wait(o_free, (items_done & 1) ^ 1, abort_flag, P.status)) break;
         tc_fence_after();
         const uint32_t q0 = smem_u32(sQ);
         bool ok = true;
@@ -332,13 +380,14 @@ __global__ void __launch_bounds__(192, 1)
           if (j >= 1) {
             // O += P_{j-1} V_{j-1}
             const uint32_t np = n + j - 1;
+            if (j == 1 && !mbar_wait(o_free, (items_done & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
             if (!mbar_wait(&p_full[np & 1], (np >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
             const int pst = (int)(np % C::STAGES);
             const uint32_t v0 = smem_u32(sStage + pst * C::STAGE_BYTES) + C::TILE_BYTES;
 #pragma unroll
             for (int k = 0; k < kTile / 16; ++k)
-              mma_ts(tO, tS[np & 1] + k * 8, sdesc_mnmajor(v0 + k * 2048, kTile * 128), C::IDESC_O,
+              mma_ts(tO, tP[np & 1] + k * 8, sdesc_mnmajor(v0 + k * 2048, kTile * 128), C::IDESC_O,
                      (j > 1 || k > 0) ? 1u : 0u);
             mma_commit(&kv_empty[pst]);
           }
@@ -355,8 +404,10 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ------------------------------------------------------------ activation + epilogue
     const int quarter = warp & 3;
+    const int wg = (warp - 2) >> 2;                 // warpgroup: key columns [64 wg, 64 wg + 64)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    constexpr uint32_t kActThreads = 32 * C::ACT_WARPS;
     uint32_t n = 0, items_done = 0;
     int cur_h = -1;
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
@@ -372,56 +423,86 @@ __global__ void __launch_bounds__(192, 1)
       const bool cand = qpos >= g.hlen;
       const long long tq = rvalid ? a.q_ts[g.qs + r0 + row] : 0;
       if (item.h != cur_h) {
-        named_barrier(1, 128);
-        if (row < 32) {
-          rab[row] = (a.rab_pos && row < a.P) ? a.rab_pos[item.h * a.P + row] : 0.f;
-          rab[32 + row] = (a.rab_time && row < a.Bt) ? a.rab_time[item.h * a.Bt + row] : 0.f;
+        named_barrier(1, kActThreads);
+        if (threadIdx.x - 64 < 32) {
+          const int t = threadIdx.x - 64;
+          rab[t] = (a.rab_pos && t < a.P) ? a.rab_pos[item.h * a.P + t] : 0.f;
+          rab[32 + t] = (a.rab_time && t < a.Bt) ? a.rab_time[item.h * a.Bt + t] : 0.f;
         }
-        named_barrier(1, 128);
+        named_barrier(1, kActThreads);
         cur_h = item.h;
       }
       bool stop = *abort_flag != 0;
-      if (named_barrier_any(1, 128, stop)) break;
+      if (named_barrier_any(1, kActThreads, stop)) break;
       bool fail = false;
+      const float rp_far = rab[a.P - 1];
       for (int j = 0; j < nk; ++j) {
         const uint32_t nj = n + j;
         const uint32_t buf = nj & 1, par = (nj >> 1) & 1;
         fail = !mbar_wait(&s_full[buf], par, abort_flag, P.status);
-        if (named_barrier_any(1, 128, fail)) { fail = true; break; }
+        if (named_barrier_any(1, kActThreads, fail)) { fail = true; break; }
         tc_fence_after();
-        // the stage holding this tile's keys (and their timestamps)
         const int kst = (int)(nj % C::STAGES);
         const long long* kts = reinterpret_cast<const long long*>(sStage + kst * C::STAGE_BYTES + C::KV_BYTES);
         const int k0 = j * kTile;
-        const bool need_mask = (k0 + kTile > kend) || (!cand && k0 + kTile - 1 > qpos) || !rvalid;
+        // fast path: every key of the tile visible, last position bucket,
+        // at most two time-bucket breakpoints along the row
+        const bool full_tile = k0 + kTile <= kend && (cand || k0 + kTile - 1 <= qpos);
+        const bool far = qp_clamped - (k0 + kTile - 1) >= a.P - 1;
+        int nb = 3, b_lo = 0;
+        if (rvalid && full_tile && far) {
+          const int b_hi = time_bucket32(tq - kts[0], a.Bt);
+          b_lo = time_bucket32(tq - kts[kTile - 1], a.Bt);
+          nb = b_hi - b_lo;
+        }
+        const bool fast = __all_sync(0xffffffffu, rvalid && full_tile && far && nb <= 2);
+        const uint32_t sbuf = tS[buf] + lane_off + wg * 64;
+        const uint32_t pbuf = tP[buf] + lane_off + wg * 32;
+        if (fast) {
+          const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)nb);
+          int p[2] = {0, 0};
+          float hd[2] = {0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) {
-          uint32_t s[32];
-          tmem_ld32(tS[buf] + lane_off + c * 32, s);
-          tmem_ld_wait();
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pv[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int col = c * 32 + e + u;
-              const int jk = k0 + col;
-              const int dp = qp_clamped - jk;
-              const int bp = min(max(dp, 0), a.P - 1);
-              const long long dt = tq - kts[col];
-              const int bt = dt <= 0 ? 0 : min(64 - __clzll(dt), a.Bt - 1);
-              float x = __uint_as_float(s[e + u]) + rab[bp] + rab[32 + bt];
-              float y = silu_fast(x);
-              if (need_mask) {
-                const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
-                y = ok ? y : 0.f;
-              }
-              pv[u] = y;
+          for (int k = 0; k < 2; ++k)
+            if (k < nb) {
+              const int b = b_lo + 1 + k;
+              p[k] = count_le128(kts, tq - (1LL << (b - 1))) - wg * 64;
+              hd[k] = 0.5f * (rab[32 + b] - rab[32 + b - 1]);
             }
-            pk[e / 2] = pack_bf16(pv[0], pv[1]);
+          const float hb = 0.5f * (rp_far + rab[32 + b_lo]);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t sv[32], pk[16];
+            tmem_ld32(sbuf + c * 32, sv);
+            tmem_ld_wait();
+            if (nbw == 0) act_chunk_fast<0>(sv, c * 32, hb, p, hd, pk);
+            else if (nbw == 1) act_chunk_fast<1>(sv, c * 32, hb, p, hd, pk);
+            else act_chunk_fast<2>(sv, c * 32, hb, p, hd, pk);
+            tmem_st16(pbuf + c * 16, pk);
           }
-          tmem_st16(tS[buf] + lane_off + c * 16, pk);
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t sv[32], pk[16];
+            tmem_ld32(sbuf + c * 32, sv);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              float y[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int col = wg * 64 + c * 32 + e + u;
+                const int jk = k0 + col;
+                const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
+                const int bp = min(max(qp_clamped - jk, 0), a.P - 1);
+                const int bt = time_bucket32(tq - kts[col], a.Bt);
+                const float h = 0.5f * (__uint_as_float(sv[e + u]) + rab[bp] + rab[32 + bt]);
+                y[u] = ok ? silu_half(h) : 0.f;
+              }
+              pk[e / 2] = pack_bf16(y[0], y[1]);
+            }
+            tmem_st16(pbuf + c * 16, pk);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -430,7 +511,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (fail) break;
       n += nk;
-      // ---- epilogue: O (fp32) = (1/N) (P V  [+ self term])
+      // ---- epilogue: this warpgroup's half of O = (1/N) (P V [+ self term])
       float* O = static_cast<float*>(a.o);
       const int h = item.h;
       float self_w = 0.f;
@@ -456,12 +537,13 @@ __global__ void __launch_bounds__(192, 1)
       if (nk > 0) {
         fail = !mbar_wait(o_full, items_done & 1, abort_flag, P.status);
         ++items_done;
-        if (named_barrier_any(1, 128, fail)) break;
+        if (named_barrier_any(1, kActThreads, fail)) break;
         tc_fence_after();
       }
       const bf16* sv = static_cast<const bf16*>(a.self_v) + (g.qs + r0 + row) * a.q_stride + h * DH;
 #pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
+      for (int cc = 0; cc < DH / 64; ++cc) {
+        const int c = wg * (DH / 64) + cc;            // 32-column chunk of O
         float o[32];
         if (nk > 0) {
           uint32_t r[32];
@@ -545,7 +627,7 @@ cudaError_t launch_fwd(const AttnArgs& a, void* ws, uint32_t* status, cudaStream
   auto kern = attn_fwd_tc_kernel<DH>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<sm_count_attn(), 192, C::SMEM, s>>>(tQ, tK, tV, P);
+  kern<<<sm_count_attn(), C::THREADS, C::SMEM, s>>>(tQ, tK, tV, P);
   count_launch();
   return cudaGetLastError();
 }

@@ -67,6 +67,7 @@ _SIGS = {
     "hstu_attention_fwd": (I32, [_CP, P, P, P, P, I32, I64, P, P, P, P, S, P]),
     "hstu_attention_fwd_cached": (I32, [_CP, P, P, P, P, I32, I64, P, P, P, I64, P, P, P, S, P]),
     "hstu_attention_workspace_size": (S, [_CP, I32, I64]),
+    "hstu_attention_fwd_noalloc": (I32, [_CP, P, P, P, P, I32, I64, P, P, P, P]),
     "hstu_ln_gate_fwd": (I32, [_CP, P, P, P, P, I64, P, P, P, P]),
     "hstu_proj_out_fwd": (I32, [_CP, P, P, P, P, I64, P, P]),
     "hstu_proj_out_bwd": (I32, [_CP, P, P, P, I64, P, P, P, P]),
@@ -249,6 +250,16 @@ def attention_fwd(cfg, rab_pos, rab_time, g, offsets, timestamps, num_targets, o
                                     ptr(offsets), B, T, ptr(timestamps), ptr(num_targets),
                                     ptr(o_out), ptr(ws), ws.numel(), stream_ptr(stream)),
            "hstu_attention_fwd")
+
+
+def attention_fwd_noalloc(cfg, rab_pos, rab_time, g, offsets, timestamps, num_targets, o_out,
+                          stream=None):
+    """hstu_attention_fwd without a workspace (static device scratch)."""
+    B, T = offsets.numel() - 1, g.shape[0]
+    _check(lib().hstu_attention_fwd_noalloc(ctypes.byref(cfg), ptr(rab_pos), ptr(rab_time), ptr(g),
+                                            ptr(offsets), B, T, ptr(timestamps), ptr(num_targets),
+                                            ptr(o_out), stream_ptr(stream)),
+           "hstu_attention_fwd_noalloc")
 
 
 def attention_fwd_cached(cfg, rab_pos, rab_time, cand_g, cand_offsets, cand_ts, hist_kv,

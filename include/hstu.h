@@ -188,6 +188,29 @@ hstu_status hstu_attention_fwd_cached(const hstu_config* cfg, const float* rab_p
                                       const int64_t* hist_timestamps, void* o_out,
                                       void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* hstu_attention_fwd for callers that cannot allocate device memory (the
+ * paper has no counterpart: this is a property of this library's interface).
+ * Same arguments and result as hstu_attention_fwd, without the workspace: the
+ * scratch (the work list of the tensor-core kernel) lives in a 2 MiB static
+ * device array that every GPU loading the library keeps until process exit.
+ * Meant for processes held to a device-memory budget fixed at start-up, which
+ * may not allocate while serving, and for C hosts that own only their input
+ * and output buffers.
+ *   - Capacity: inputs whose work list exceeds the array (about 260,000
+ *     (128-query tile, head) items, i.e. roughly (T / 128 + B) * H <= 262,000)
+ *     return HSTU_ERR_WORKSPACE; nothing is launched.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - It never calls cudaMalloc, cudaFree or any allocating routine.
+ *   - Every call on a device shares the same array and rebuilds (and clears)
+ *     its contents; calls that can overlap on the GPU (other streams, other
+ *     host threads) race on it and must be serialised by the caller. */
+hstu_status hstu_attention_fwd_noalloc(const hstu_config* cfg, const float* rab_pos,
+                                       const float* rab_time, const void* g,
+                                       const int64_t* seq_offsets, int32_t B, int64_t T,
+                                       const int64_t* timestamps, const int32_t* num_targets,
+                                       void* o_out, cudaStream_t stream);
+
 /* Bytes of workspace the attention entry points need. Host only. */
 size_t hstu_attention_workspace_size(const hstu_config* cfg, int32_t B, int64_t T);
 

@@ -627,6 +627,495 @@ __global__ void __launch_bounds__(kBThreads, 1)
   }
 }
 
+int sms();
+
+// ---------------------------------------------------------------------------
+// Pipelined backward for dh = 128: 64-query blocks
+// ---------------------------------------------------------------------------
+// With 64-query blocks two S^T/dP^T buffer pairs (4 x 64 TMEM columns) fit
+// next to the resident dV and dK accumulators (2 x 128), so the MMA thread
+// issues block g's S^T = K Q_g^T and dP^T = V dO_g^T before it waits for the
+// activation of block g-1, whose dV, dK and dQ^T MMAs then overlap the
+// activation of block g.  dQ^T_g = K^T dS_g (M = dh rows, 64 query columns)
+// goes into block g's S^T columns once dV has read P^T from them; the
+// activation warps drain it one block behind: transposed into a dense 64 x 128
+// fp32 tile in shared memory and added to the fp32 dQ accumulator with one TMA
+// bulk reduce-add (rows past the sequence end carry exact zeros).  Q/dO
+// blocks come through a two-stage ring.
+// TMEM: S^T_0 [0,64) dP^T_0 [64,128) S^T_1 [128,192) dP^T_1 [192,256)
+//       dV [256,384) dK [384,512)
+constexpr int kQB = 64;
+constexpr int kQStages = 2;
+
+struct B3Cfg {
+  static constexpr int DH = 128;
+  static constexpr int KTILE = kT * DH * 2;            // 128 keys x 128 bf16 = 32 KB
+  static constexpr int QTILE = kQB * DH * 2;           // 64 queries x 128 bf16 = 16 KB
+  static constexpr int QSTAGE = 2 * QTILE + 1024;      // Q, dO, timestamps (64 x 8 B, padded)
+  static constexpr int DS_BYTES = kT * kQB * 2;        // dS [key][query] for one block = 16 KB
+  static constexpr int DQ_BYTES = kQB * DH * 4;        // dQ staging [query][dh] fp32 = 32 KB
+  static constexpr int SMEM = 1024 + 2 * KTILE + kQStages * QSTAGE + 2 * DS_BYTES + DQ_BYTES + 2048;
+  static constexpr uint32_t IDESC_ST = idesc_bf16(128, kQB, false, false);   // K Q^T, V dO^T
+  static constexpr uint32_t IDESC_DKV = idesc_bf16(128, DH, false, true);    // P^T dO, dS^T Q
+  static constexpr uint32_t IDESC_DQT = idesc_bf16(128, kQB, true, true);    // K^T dS^T
+};
+
+// query blocks that see key tile kt: from its first key to the end
+__device__ __forceinline__ int qblocks(int n, int kt) { return (n - kt * kT + kQB - 1) / kQB; }
+
+__global__ void __launch_bounds__(kBThreads, 1)
+    attn_bwd_tc3_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                        const __grid_constant__ CUtensorMap tmdQ, const BParams P) {
+  using C = B3Cfg;
+  constexpr int DH = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + C::KTILE;
+  uint8_t* sQD = sV + C::KTILE;                    // kQStages x (Q | dO | timestamps)
+  uint8_t* sDS = sQD + kQStages * C::QSTAGE;        // 2 x dS
+  float* sDQ = reinterpret_cast<float*>(sDS + 2 * C::DS_BYTES);   // dQ staging [64][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + 2 * C::DS_BYTES + C::DQ_BYTES);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* qd_full = bars + 2;                     // [3]
+  uint64_t* qd_empty = bars + 5;                    // [3]
+  uint64_t* st_full = bars + 8;                     // [2]
+  uint64_t* pds_full = bars + 10;                   // [2] (8 warps)
+  uint64_t* dq_full = bars + 12;                    // [2]
+  uint64_t* a_free = bars + 14;                     // [2] (8 warps)
+  uint64_t* dkv_full = bars + 16;
+  uint64_t* dkv_free = bars + 17;                   // (8 warps)
+  uint64_t* done_bar = bars + 18;
+  float* rab = reinterpret_cast<float*>(bars + 20);  // [64]
+  float* drab = rab + 64;                            // [64]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drab + 64);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const AttnArgs& a = P.A.f;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int total = *P.w.total;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 19; ++i) {
+      const bool act = (i == 10 || i == 11 || i == 14 || i == 15 || i == 17);
+      mbar_init(&bars[i], act ? kActWarps : 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS[2] = {tmem, tmem + 128}, tD[2] = {tmem + 64, tmem + 192};
+  const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t items_done = 0, g = 0;
+    bool kv_iss = false;
+    uint32_t kv_par = 0, issued = 0, issued_par = 0;
+    for (int it = blockIdx.x; it < total; it += gridDim.x) {
+      if (*abort_flag) break;
+      const BItem item = P.w.items[it];
+      int64_t s0;
+      int n, hlen;
+      bgeom(a, item.b, s0, n, hlen);
+      const int k0 = item.kt * kT;
+      const int nqb = qblocks(n, item.kt);
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(kv_empty, (items_done & 1) ^ 1, abort_flag, P.status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_expect_tx(kv_full, 2 * C::KTILE);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          tma_load_2d(sK + x * (kT * 128), &tmK, kv_full, item.h * DH + 64 * x, (int32_t)(s0 + k0));
+          tma_load_2d(sV + x * (kT * 128), &tmV, kv_full, item.h * DH + 64 * x, (int32_t)(s0 + k0));
+        }
+        kv_iss = true;
+        kv_par = items_done & 1;
+      }
+      ++items_done;
+      for (int m = 0; m < nqb; ++m, ++g) {
+        const int st = (int)(g % kQStages);
+        const uint32_t par = (g / kQStages) & 1;
+        const int q0 = k0 + m * kQB;
+        if (lane == 0) ok = mbar_wait(&qd_empty[st], par ^ 1, abort_flag, P.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        uint8_t* stg = sQD + st * C::QSTAGE;
+        long long* qts = reinterpret_cast<long long*>(stg + 2 * C::QTILE);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = lane + 32 * u;
+          // past the sequence: a large sentinel keeps the staged times sorted
+          qts[c] = (q0 + c < n) ? a.q_ts[s0 + q0 + c] : (1LL << 62);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_expect_tx(&qd_full[st], 2 * C::QTILE);
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            tma_load_2d(stg + x * (kQB * 128), &tmQ, &qd_full[st], item.h * DH + 64 * x, (int32_t)(s0 + q0));
+            tma_load_2d(stg + C::QTILE + x * (kQB * 128), &tmdO, &qd_full[st], item.h * DH + 64 * x,
+                        (int32_t)(s0 + q0));
+          }
+          issued |= 1u << st;
+          issued_par = (issued_par & ~(1u << st)) | (par << st);
+        }
+      }
+      if (!ok) break;
+    }
+    if (lane == 0) {
+      volatile int never = 0;
+      if (kv_iss) mbar_wait(kv_full, kv_par, &never, P.status);
+      for (int s2 = 0; s2 < kQStages; ++s2)
+        if (issued & (1u << s2)) mbar_wait(&qd_full[s2], (issued_par >> s2) & 1u, &never, P.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t items_done = 0, g = 0;
+      const uint32_t k_s = smem_u32(sK), v_s = smem_u32(sV);
+      for (int it = blockIdx.x; it < total; it += gridDim.x) {
+        if (*abort_flag) break;
+        const BItem item = P.w.items[it];
+        int64_t s0;
+        int n, hlen;
+        bgeom(a, item.b, s0, n, hlen);
+        const int nqb = qblocks(n, item.kt);
+        if (!mbar_wait(kv_full, items_done & 1, abort_flag, P.status)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int m = 0; m <= nqb && ok; ++m) {
+          if (m < nqb) {
+            // block g + m: S^T, dP^T into buffer (g + m) & 1
+            const uint32_t gb = g + m, b = gb & 1;
+            const int st = (int)(gb % kQStages);
+            if (!mbar_wait(&qd_full[st], (gb / kQStages) & 1, abort_flag, P.status)) { ok = false; break; }
+            if (gb >= 2 && !mbar_wait(&a_free[b], ((gb - 2) >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t q_s = smem_u32(sQD + st * C::QSTAGE), do_s = q_s + C::QTILE;
+#pragma unroll
+            for (int k = 0; k < DH / 16; ++k) {
+              const uint32_t koff = (k / 4) * (kT * 128) + (k % 4) * 32;
+              const uint32_t qoff = (k / 4) * (kQB * 128) + (k % 4) * 32;
+              mma_ss(tS[b], sdesc_kmajor(k_s + koff), sdesc_kmajor(q_s + qoff), C::IDESC_ST, k > 0);
+            }
+#pragma unroll
+            for (int k = 0; k < DH / 16; ++k) {
+              const uint32_t koff = (k / 4) * (kT * 128) + (k % 4) * 32;
+              const uint32_t qoff = (k / 4) * (kQB * 128) + (k % 4) * 32;
+              mma_ss(tD[b], sdesc_kmajor(v_s + koff), sdesc_kmajor(do_s + qoff), C::IDESC_ST, k > 0);
+            }
+            mma_commit(&st_full[b]);
+          }
+          if (m >= 1) {
+            // block g + m - 1: dV, dK accumulate; dQ^T into its S^T columns
+            const uint32_t gp = g + m - 1, b = gp & 1;
+            const int st = (int)(gp % kQStages);
+            if (m == 1 && !mbar_wait(dkv_free, (items_done & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
+            if (!mbar_wait(&pds_full[b], (gp >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t q_s = smem_u32(sQD + st * C::QSTAGE), do_s = q_s + C::QTILE;
+            const uint32_t acc0 = m > 1 ? 1u : 0u;
+            // A operand halves: queries [0,32) at columns [0,16), [32,64) at [32,48)
+#pragma unroll
+            for (int k = 0; k < kQB / 16; ++k)
+              mma_ts(tdV, tS[b] + (k / 2) * 32 + (k % 2) * 8, sdesc_mnmajor(do_s + k * 2048, kQB * 128),
+                     C::IDESC_DKV, (acc0 || k > 0) ? 1u : 0u);
+#pragma unroll
+            for (int k = 0; k < kQB / 16; ++k)
+              mma_ts(tdK, tD[b] + (k / 2) * 32 + (k % 2) * 8, sdesc_mnmajor(q_s + k * 2048, kQB * 128),
+                     C::IDESC_DKV, (acc0 || k > 0) ? 1u : 0u);
+            mma_commit(&qd_empty[st]);
+            const uint32_t ds_s = smem_u32(sDS + b * C::DS_BYTES);
+#pragma unroll
+            for (int k = 0; k < kT / 16; ++k)
+              mma_ss(tS[b], sdesc_mnmajor(k_s + k * 2048, kT * 128), sdesc_mnmajor(ds_s + k * 2048, kT * 128),
+                     C::IDESC_DQT, k > 0 ? 1u : 0u);
+            mma_commit(&dq_full[b]);
+          }
+        }
+        if (!ok) break;
+        g += nqb;
+        ++items_done;
+        mma_commit(kv_empty);
+        mma_commit(dkv_full);
+      }
+      mma_commit(done_bar);
+      volatile int never = 0;
+      mbar_wait(done_bar, 0, &never, P.status);
+    }
+  } else {
+    // ------------------------------------------------------------ key-row warps
+    const int quarter = warp & 3;
+    const int wg = (warp - 2) >> 2;                  // query columns [32 wg, 32 wg + 32) of a block
+    const int row = quarter * 32 + lane;             // key in the tile (S^T lane) / dh row (dQ^T lane)
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    constexpr uint32_t kAct = 32 * kActWarps;
+    const int d = P.A.d;
+    uint32_t items_done = 0, g = 0;
+    int cur_h = -1;
+    const float inv_N = a.inv_N;
+    const int ti = threadIdx.x - 64;
+    bool fail = false;
+    for (int it = blockIdx.x; it < total && !fail; it += gridDim.x) {
+      const BItem item = P.w.items[it];
+      int64_t s0;
+      int n, hlen;
+      bgeom(a, item.b, s0, n, hlen);
+      const int k0 = item.kt * kT;
+      const int nqb = qblocks(n, item.kt);
+      const int jk = k0 + row;
+      const bool kvalid = jk < hlen;
+      const long long tk = kvalid ? a.kv_ts[s0 + jk] : 0;
+      if (item.h != cur_h) {
+        named_barrier(1, kAct);
+        if (cur_h >= 0 && ti < 64) {
+          float* dst = ti < 32 ? P.A.drab_pos : P.A.drab_time;
+          const int nb = ti < 32 ? a.P : a.Bt;
+          const int bi = ti & 31;
+          if (dst && bi < nb && drab[ti] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[ti] * inv_N);
+        }
+        if (ti < 32) {
+          rab[ti] = (a.rab_pos && ti < a.P) ? a.rab_pos[item.h * a.P + ti] : 0.f;
+          rab[32 + ti] = (a.rab_time && ti < a.Bt) ? a.rab_time[item.h * a.Bt + ti] : 0.f;
+        }
+        if (ti < 64) drab[ti] = 0.f;
+        named_barrier(1, kAct);
+        cur_h = item.h;
+      }
+      if (named_barrier_any(1, kAct, *abort_flag != 0)) { fail = true; break; }
+      const float rp_far = rab[a.P - 1];
+      // dS sums per rab bucket of this key row: the last position bucket in a
+      // register, the others and the time buckets run-length encoded (both
+      // buckets are non-decreasing along the row's queries), flushed to
+      // shared memory only when the bucket changes and at the item's end
+      float far_sum = 0.f, p_sum = 0.f, t_sum = 0.f;
+      int pb_cur = -1, tb_cur = -1;
+      auto add_t = [&](int bkt, float v) {
+        if (bkt != tb_cur) {
+          if (tb_cur >= 0) atomicAdd(&drab[32 + tb_cur], t_sum);
+          tb_cur = bkt;
+          t_sum = 0.f;
+        }
+        t_sum += v;
+      };
+      auto add_p = [&](int bkt, float v) {
+        if (bkt == a.P - 1) {
+          far_sum += v;
+          return;
+        }
+        if (bkt != pb_cur) {
+          if (pb_cur >= 0) atomicAdd(&drab[pb_cur], p_sum);
+          pb_cur = bkt;
+          p_sum = 0.f;
+        }
+        p_sum += v;
+      };
+      // drain dQ^T of block gd (query rows q0d ..): free its TMEM columns,
+      // transpose into the staging tile, one bulk reduce-add into dQ
+      auto drain = [&](uint32_t gd, int q0d) -> bool {
+        const uint32_t b = gd & 1;
+        bool f = !mbar_wait(&dq_full[b], (gd >> 1) & 1, abort_flag, P.status);
+        if (ti == 0) bulk_wait_read0();             // the previous reduce has read the staging tile
+        if (named_barrier_any(1, kAct, f)) return false;
+        tc_fence_after();
+        uint32_t r[32];
+        tmem_ld32(tS[b] + lane_off + wg * 32, r);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_free[b]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sDQ[(wg * 32 + i) * DH + row] = __uint_as_float(r[i]) * inv_N;
+        fence_proxy_async_smem();
+        named_barrier(1, kAct);
+        if (ti == 0) {
+          tma_reduce_add_2d(&tmdQ, sDQ, item.h * DH, (int32_t)(s0 + q0d));
+          bulk_commit();
+        }
+        return true;
+      };
+
+      for (int m = 0; m < nqb; ++m) {
+        const uint32_t gb = g + m, b = gb & 1;
+        const int st = (int)(gb % kQStages);
+        const int q0 = k0 + m * kQB;
+        fail = !mbar_wait(&st_full[b], (gb >> 1) & 1, abort_flag, P.status);
+        if (named_barrier_any(1, kAct, fail)) { fail = true; break; }
+        tc_fence_after();
+        const long long* qts = reinterpret_cast<const long long*>(sQD + st * C::QSTAGE + 2 * C::QTILE);
+        const int qf = q0 + wg * 32;                 // first query of this warpgroup's 32
+        const bool full = kvalid && qf + 31 < n && jk <= qf;
+        const bool far = min(qf, hlen) - jk >= a.P - 1;
+        int nb = 3, b_lo = 0;
+        if (full && far) {
+          b_lo = tb64(qts[wg * 32] - tk, a.Bt);
+          nb = tb64(qts[wg * 32 + 31] - tk, a.Bt) - b_lo;
+        }
+        const bool fast = __all_sync(0xffffffffu, full && far && nb <= 2);
+        uint32_t sr[32], dr[32], pk[16], dk[16];
+        tmem_ld32(tS[b] + lane_off + wg * 32, sr);
+        tmem_ld32(tD[b] + lane_off + wg * 32, dr);
+        tmem_ld_wait();
+        if (fast) {
+          const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)nb);
+          int p[2] = {32, 32};
+          float hd[2] = {0.f, 0.f};
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+            if (k < nb) {
+              const int bb = b_lo + 1 + k;
+              // this half's queries (sorted) with t <= tk + 2^(bb-1) - 1
+              const long long tau = tk + (1LL << (bb - 1)) - 1;
+              const longlong2* q2 = reinterpret_cast<const longlong2*>(qts + wg * 32);
+              int cnt = 0;
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                const longlong2 v = q2[c];
+                cnt += (v.x <= tau) + (v.y <= tau);
+              }
+              p[k] = cnt;
+              hd[k] = 0.5f * (rab[32 + bb] - rab[32 + bb - 1]);
+            }
+          const float hb = 0.5f * (rp_far + rab[32 + b_lo]);
+          float tot = 0.f, suf[2] = {0.f, 0.f};
+          if (nbw == 0) bwd_chunk_fast<0>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
+          else if (nbw == 1) bwd_chunk_fast<1>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
+          else bwd_chunk_fast<2>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
+          far_sum += tot;
+          float below = tot;
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+            if (k < nb) {
+              add_t(b_lo + k, below - suf[k]);
+              below = suf[k];
+            }
+          add_t(b_lo + nb, below);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int col = wg * 32 + e + u;
+              const int qpos = q0 + col;
+              const bool ok = kvalid && qpos < n && (qpos >= hlen || jk <= qpos);
+              float pa = 0.f, ds = 0.f;
+              if (ok) {
+                const int bp = min(max(min(qpos, hlen) - jk, 0), a.P - 1);
+                const int bt = tb64(qts[col] - tk, a.Bt);
+                const float h = 0.5f * (__uint_as_float(sr[e + u]) + rab[bp] + rab[32 + bt]);
+                const float t = tanh_fast(h);
+                const float sg = fmaf(t, 0.5f, 0.5f);
+                pa = fmaf(h, t, h);
+                ds = __uint_as_float(dr[e + u]) * fmaf(sg, fmaf(-h, t, h), sg);
+                add_p(bp, ds);
+                add_t(bt, ds);
+              }
+              pv[u] = pa;
+              dv[u] = ds;
+            }
+            pk[e / 2] = pack_bf16(pv[0], pv[1]);
+            dk[e / 2] = pack_bf16(dv[0], dv[1]);
+          }
+        }
+        tmem_st16(tS[b] + lane_off + wg * 32, pk);
+        tmem_st16(tD[b] + lane_off + wg * 32, dk);
+        uint8_t* dsb = sDS + b * C::DS_BYTES;
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          const uint4 v = make_uint4(dk[4 * g8], dk[4 * g8 + 1], dk[4 * g8 + 2], dk[4 * g8 + 3]);
+          *reinterpret_cast<uint4*>(dsb + mn_off(row, wg * 32 + g8 * 8, kT * 128)) = v;
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pds_full[b]);
+        if (m >= 1 && !drain(gb - 1, q0 - kQB)) { fail = true; break; }
+      }
+      if (fail) break;
+      if (nqb >= 1 && !drain(g + nqb - 1, k0 + (nqb - 1) * kQB)) { fail = true; break; }
+      // flush this key row's bucket sums
+      if (tb_cur >= 0) atomicAdd(&drab[32 + tb_cur], t_sum);
+      if (pb_cur >= 0) atomicAdd(&drab[pb_cur], p_sum);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) far_sum += __shfl_xor_sync(0xffffffffu, far_sum, o);
+      if (lane == 0 && far_sum != 0.f) atomicAdd(&drab[a.P - 1], far_sum);
+      g += nqb;
+      // this warpgroup's half of dK, dV (times 1/N and SiLU'(Pre)) into dPre
+      fail = !mbar_wait(dkv_full, items_done & 1, abort_flag, P.status);
+      ++items_done;
+      if (named_barrier_any(1, kAct, fail)) { fail = true; break; }
+      tc_fence_after();
+      const bf16* pre = static_cast<const bf16*>(P.A.pre);
+      bf16* dpre = static_cast<bf16*>(P.A.dpre);
+      const int64_t rowoff = (s0 + jk) * P.A.pre_stride;
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = wg * 2 + cc;
+        uint32_t rv[32], rk[32];
+        tmem_ld32(tdV + lane_off + c * 32, rv);
+        tmem_ld32(tdK + lane_off + c * 32, rk);
+        tmem_ld_wait();
+        if (kvalid) {
+          const int col = item.h * DH + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            const uint4 pv4 = *reinterpret_cast<const uint4*>(pre + rowoff + d + col + i);
+            const uint4 pk4 = *reinterpret_cast<const uint4*>(pre + rowoff + 3 * d + col + i);
+            const __nv_bfloat162* pvh = reinterpret_cast<const __nv_bfloat162*>(&pv4);
+            const __nv_bfloat162* pkh = reinterpret_cast<const __nv_bfloat162*>(&pk4);
+            uint4 ov, ok4;
+            uint32_t* ovw = reinterpret_cast<uint32_t*>(&ov);
+            uint32_t* okw = reinterpret_cast<uint32_t*>(&ok4);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 fv = __bfloat1622float2(pvh[u]);
+              const float2 fk = __bfloat1622float2(pkh[u]);
+              ovw[u] = pack_bf16(__uint_as_float(rv[i + 2 * u]) * inv_N * silu_grad_acc(fv.x),
+                                 __uint_as_float(rv[i + 2 * u + 1]) * inv_N * silu_grad_acc(fv.y));
+              okw[u] = pack_bf16(__uint_as_float(rk[i + 2 * u]) * inv_N * silu_grad_acc(fk.x),
+                                 __uint_as_float(rk[i + 2 * u + 1]) * inv_N * silu_grad_acc(fk.y));
+            }
+            *reinterpret_cast<uint4*>(dpre + rowoff + d + col + i) = ov;
+            *reinterpret_cast<uint4*>(dpre + rowoff + 3 * d + col + i) = ok4;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dkv_free);
+    }
+    // flush the last head's bucket sums
+    named_barrier(1, kAct);
+    if (cur_h >= 0 && ti < 64) {
+      float* dst = ti < 32 ? P.A.drab_pos : P.A.drab_time;
+      const int nb = ti < 32 ? a.P : a.Bt;
+      const int bi = ti & 31;
+      if (dst && bi < nb && drab[ti] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[ti] * inv_N);
+    }
+    if (ti == 0) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_bwd3(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaStream_t s);
+
 int sms() {
   static int n = 0;
   if (n == 0) {
@@ -669,6 +1158,38 @@ cudaError_t launch_bwd(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaStr
   return cudaGetLastError();
 }
 
+cudaError_t launch_bwd3(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaStream_t s) {
+  using C = B3Cfg;
+  const AttnArgs& a = A.f;
+  const int d = a.H * 128;
+  CUtensorMap tQ, tK, tV, tdO;
+  bool ok = encode_tmap_2d(&tQ, false, a.q, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)a.q_stride, 64, kQB) &&
+            encode_tmap_2d(&tK, false, a.k, (uint64_t)d, (uint64_t)a.kv_rows, (uint64_t)a.kv_stride, 64, kT) &&
+            encode_tmap_2d(&tV, false, a.v, (uint64_t)d, (uint64_t)a.kv_rows, (uint64_t)a.kv_stride, 64, kT) &&
+            encode_tmap_2d(&tdO, false, A.dout, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)a.o_stride, 64, kQB);
+  CUtensorMap tdQ;  // fp32 [T][d] accumulator, dense 128 x 64 boxes, no swizzle
+  ok = ok && encode_tmap_2d(&tdQ, true, A.dq_acc, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)A.d, 128, kQB,
+                            false);
+  if (!ok) return cudaErrorInvalidValue;
+  BSched w = bsched(ws);
+  cudaError_t e = cudaMemsetAsync(w.hist, 0, 3 * kMaxCostB * sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
+  const int blocks = (a.B + 255) / 256;
+  bsched_count<<<blocks, 256, 0, s>>>(a, w);
+  bsched_scan<<<1, 32, 0, s>>>(w);
+  bsched_fill<<<blocks, 256, 0, s>>>(a, w);
+  count_launch(3);
+  BParams P;
+  P.A = A;
+  P.w = w;
+  P.status = status;
+  e = cudaFuncSetAttribute(attn_bwd_tc3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  attn_bwd_tc3_kernel<<<sms(), kBThreads, C::SMEM, s>>>(tQ, tK, tV, tdO, tdQ, P);
+  count_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t attn_bwd_sched_bytes(int B, int64_t T, int H) {
@@ -684,7 +1205,7 @@ bool attention_bwd_tc_supported(int dtype, const AttnBwdArgs& A) {
 }
 
 cudaError_t attention_bwd_tc(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaStream_t s) {
-  if (A.f.dh == 128) return launch_bwd<128>(A, ws, status, s);
+  if (A.f.dh == 128) return launch_bwd3(A, ws, status, s);
   return launch_bwd<64>(A, ws, status, s);
 }
 

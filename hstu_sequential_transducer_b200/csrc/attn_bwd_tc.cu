@@ -144,6 +144,7 @@ __device__ __forceinline__ float tanh_fast(float x) {
 }
 
 constexpr int kBThreads = 320;
+constexpr int kPrefetch = 4;   // query blocks the backward producer prefetches ahead
 constexpr int kActWarps = 8;
 
 __device__ __forceinline__ int tb64(long long dt, int Bt) {
@@ -158,6 +159,15 @@ __device__ __forceinline__ int count_le_128(const long long* cts, long long tau)
   for (int step = 64; step >= 1; step >>= 1)
     if (cts[lo + step - 1] <= tau) lo += step;
   return lo;
+}
+
+// Number of the 32 non-decreasing values cts[] that are <= tau.
+__device__ __forceinline__ int count_le_32(const long long* cts, long long tau) {
+  int lo = 0;
+#pragma unroll
+  for (int step = 16; step >= 1; step >>= 1)
+    if (cts[lo + step - 1] <= tau) lo += step;
+  return lo + (cts[lo] <= tau ? 1 : 0);
 }
 
 // One 32-column chunk of the fast path: h = S/2 + bias/2 where columns
@@ -638,23 +648,30 @@ int sms();
 // activation of block g-1, whose dV, dK and dQ^T MMAs then overlap the
 // activation of block g.  dQ^T_g = K^T dS_g (M = dh rows, 64 query columns)
 // goes into block g's S^T columns once dV has read P^T from them; the
-// activation warps drain it one block behind: transposed into a dense 64 x 128
-// fp32 tile in shared memory and added to the fp32 dQ accumulator with one TMA
-// bulk reduce-add (rows past the sequence end carry exact zeros).  Q/dO
-// blocks come through a two-stage ring.
+// activation warps drain it one block behind: each warpgroup transposes its
+// 32 queries into a dense 32 x 128 fp32 tile in shared memory and adds it to
+// the fp32 dQ accumulator with one TMA bulk reduce-add (rows past the
+// sequence end carry exact zeros).  Q/dO blocks come through a three-stage
+// ring, so that the loads of block g+1 are in flight while block g-1's dV and
+// dK still read their stage; the block times have a ring of their own.  This
+// packs the whole 227 KB budget, so the kernel relies on a 1024-byte aligned
+// dynamic shared memory base (checked; it reports kStatusSmemAlign if not).
 // TMEM: S^T_0 [0,64) dP^T_0 [64,128) S^T_1 [128,192) dP^T_1 [192,256)
 //       dV [256,384) dK [384,512)
 constexpr int kQB = 64;
-constexpr int kQStages = 2;
+constexpr int kQStages = 3;
 
 struct B3Cfg {
   static constexpr int DH = 128;
   static constexpr int KTILE = kT * DH * 2;            // 128 keys x 128 bf16 = 32 KB
   static constexpr int QTILE = kQB * DH * 2;           // 64 queries x 128 bf16 = 16 KB
-  static constexpr int QSTAGE = 2 * QTILE + 1024;      // Q, dO, timestamps (64 x 8 B, padded)
+  static constexpr int QSTAGE = 2 * QTILE;             // Q, dO
+  static constexpr int TS_BYTES = kQB * 8;             // one block's times
   static constexpr int DS_BYTES = kT * kQB * 2;        // dS [key][query] for one block = 16 KB
-  static constexpr int DQ_BYTES = kQB * DH * 4;        // dQ staging [query][dh] fp32 = 32 KB
-  static constexpr int SMEM = 1024 + 2 * KTILE + kQStages * QSTAGE + 2 * DS_BYTES + DQ_BYTES + 2048;
+  static constexpr int DQ_BYTES = kQB * DH * 4;        // dQ staging, 2 x [32 queries][dh] fp32 = 32 KB
+  static constexpr int BAR_BYTES = 1536;               // barriers, rab tables, TMEM slot
+  static constexpr int SMEM = 2 * KTILE + kQStages * QSTAGE + 2 * DS_BYTES + DQ_BYTES + kQStages * TS_BYTES +
+                              BAR_BYTES;
   static constexpr uint32_t IDESC_ST = idesc_bf16(128, kQB, false, false);   // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DKV = idesc_bf16(128, DH, false, true);    // P^T dO, dS^T Q
   static constexpr uint32_t IDESC_DQT = idesc_bf16(128, kQB, true, true);    // K^T dS^T
@@ -668,15 +685,21 @@ __global__ void __launch_bounds__(kBThreads, 1)
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                         const __grid_constant__ CUtensorMap tmdQ, const BParams P) {
   using C = B3Cfg;
+  static_assert(C::SMEM <= 232448, "shared memory budget");
   constexpr int DH = 128;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {              // uniform over the block: all threads leave
+    if (threadIdx.x == 0 && P.status) atomicOr(P.status, kStatusSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::KTILE;
-  uint8_t* sQD = sV + C::KTILE;                    // kQStages x (Q | dO | timestamps)
+  uint8_t* sQD = sV + C::KTILE;                    // kQStages x (Q | dO)
   uint8_t* sDS = sQD + kQStages * C::QSTAGE;        // 2 x dS
-  float* sDQ = reinterpret_cast<float*>(sDS + 2 * C::DS_BYTES);   // dQ staging [64][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + 2 * C::DS_BYTES + C::DQ_BYTES);
+  float* sDQ = reinterpret_cast<float*>(sDS + 2 * C::DS_BYTES);   // 2 x dQ staging [32][128]
+  uint8_t* sTS = sDS + 2 * C::DS_BYTES + C::DQ_BYTES;             // kQStages x times
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sTS + kQStages * C::TS_BYTES);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
   uint64_t* qd_full = bars + 2;                     // [3]
@@ -688,9 +711,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
   uint64_t* dkv_full = bars + 16;
   uint64_t* dkv_free = bars + 17;                   // (8 warps)
   uint64_t* done_bar = bars + 18;
-  float* rab = reinterpret_cast<float*>(bars + 20);  // [64]
-  float* drab = rab + 64;                            // [64]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drab + 64);
+  float* rab = reinterpret_cast<float*>(bars + 20);  // [2][64] per warpgroup
+  float* drab = rab + 128;                           // [2][64] per warpgroup
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drab + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const AttnArgs& a = P.A.f;
@@ -710,7 +733,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128}, tD[2] = {tmem + 64, tmem + 192};
+  // S^T (then P^T, then dQ^T) of buffer b at columns 128 b, dP^T (then dS^T) at 128 b + 64
+  auto tS = [tmem](uint32_t b) { return tmem + b * 128u; };
+  auto tD = [tmem](uint32_t b) { return tmem + b * 128u + 64u; };
   const uint32_t tdV = tmem + 256, tdK = tmem + 384;
 
   if (warp == 0) {
@@ -741,21 +766,40 @@ __global__ void __launch_bounds__(kBThreads, 1)
         kv_par = items_done & 1;
       }
       ++items_done;
+      // L2 prefetch keeps the Q, dO and time rows kPrefetch blocks ahead of
+      // the loads, so that a freed stage refills at L2 rather than HBM latency
+      auto prefetch = [&](int mp) {
+        const int qp = k0 + mp * kQB;
+        if (mp >= nqb || qp >= n) return;
+        if (lane < 4) {
+          const CUtensorMap* tm = (lane & 2) ? &tmdO : &tmQ;
+          tma_prefetch_2d(tm, item.h * DH + 64 * (lane & 1), (int32_t)(s0 + qp));
+        } else if (lane < 9) {
+          const int r = qp + (lane - 4) * 16;       // 16 times of 8 bytes per 128-byte line
+          if (r < n) prefetch_l2(a.q_ts + s0 + r);
+        }
+      };
+      for (int mp = 1; mp < kPrefetch; ++mp) prefetch(mp);
       for (int m = 0; m < nqb; ++m, ++g) {
         const int st = (int)(g % kQStages);
         const uint32_t par = (g / kQStages) & 1;
         const int q0 = k0 + m * kQB;
+        prefetch(m + kPrefetch);
+        // the block's times, read while the stage is still in use; past the
+        // sequence a large sentinel keeps the staged times sorted
+        long long tq[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = lane + 32 * u;
+          tq[u] = (q0 + c < n) ? a.q_ts[s0 + q0 + c] : (1LL << 62);
+        }
         if (lane == 0) ok = mbar_wait(&qd_empty[st], par ^ 1, abort_flag, P.status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         uint8_t* stg = sQD + st * C::QSTAGE;
-        long long* qts = reinterpret_cast<long long*>(stg + 2 * C::QTILE);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = lane + 32 * u;
-          // past the sequence: a large sentinel keeps the staged times sorted
-          qts[c] = (q0 + c < n) ? a.q_ts[s0 + q0 + c] : (1LL << 62);
-        }
+        long long* qts = reinterpret_cast<long long*>(sTS + st * C::TS_BYTES);
+        qts[lane] = tq[0];
+        qts[lane + 32] = tq[1];
         __syncwarp();
         if (lane == 0) {
           mbar_expect_tx(&qd_full[st], 2 * C::QTILE);
@@ -805,13 +849,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
             for (int k = 0; k < DH / 16; ++k) {
               const uint32_t koff = (k / 4) * (kT * 128) + (k % 4) * 32;
               const uint32_t qoff = (k / 4) * (kQB * 128) + (k % 4) * 32;
-              mma_ss(tS[b], sdesc_kmajor(k_s + koff), sdesc_kmajor(q_s + qoff), C::IDESC_ST, k > 0);
+              mma_ss(tS(b), sdesc_kmajor(k_s + koff), sdesc_kmajor(q_s + qoff), C::IDESC_ST, k > 0);
             }
 #pragma unroll
             for (int k = 0; k < DH / 16; ++k) {
               const uint32_t koff = (k / 4) * (kT * 128) + (k % 4) * 32;
               const uint32_t qoff = (k / 4) * (kQB * 128) + (k % 4) * 32;
-              mma_ss(tD[b], sdesc_kmajor(v_s + koff), sdesc_kmajor(do_s + qoff), C::IDESC_ST, k > 0);
+              mma_ss(tD(b), sdesc_kmajor(v_s + koff), sdesc_kmajor(do_s + qoff), C::IDESC_ST, k > 0);
             }
             mma_commit(&st_full[b]);
           }
@@ -827,17 +871,17 @@ __global__ void __launch_bounds__(kBThreads, 1)
             // A operand halves: queries [0,32) at columns [0,16), [32,64) at [32,48)
 #pragma unroll
             for (int k = 0; k < kQB / 16; ++k)
-              mma_ts(tdV, tS[b] + (k / 2) * 32 + (k % 2) * 8, sdesc_mnmajor(do_s + k * 2048, kQB * 128),
+              mma_ts(tdV, tS(b) + (k / 2) * 32 + (k % 2) * 8, sdesc_mnmajor(do_s + k * 2048, kQB * 128),
                      C::IDESC_DKV, (acc0 || k > 0) ? 1u : 0u);
 #pragma unroll
             for (int k = 0; k < kQB / 16; ++k)
-              mma_ts(tdK, tD[b] + (k / 2) * 32 + (k % 2) * 8, sdesc_mnmajor(q_s + k * 2048, kQB * 128),
+              mma_ts(tdK, tD(b) + (k / 2) * 32 + (k % 2) * 8, sdesc_mnmajor(q_s + k * 2048, kQB * 128),
                      C::IDESC_DKV, (acc0 || k > 0) ? 1u : 0u);
             mma_commit(&qd_empty[st]);
             const uint32_t ds_s = smem_u32(sDS + b * C::DS_BYTES);
 #pragma unroll
             for (int k = 0; k < kT / 16; ++k)
-              mma_ss(tS[b], sdesc_mnmajor(k_s + k * 2048, kT * 128), sdesc_mnmajor(ds_s + k * 2048, kT * 128),
+              mma_ss(tS(b), sdesc_mnmajor(k_s + k * 2048, kT * 128), sdesc_mnmajor(ds_s + k * 2048, kT * 128),
                      C::IDESC_DQT, k > 0 ? 1u : 0u);
             mma_commit(&dq_full[b]);
           }
@@ -858,12 +902,16 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const int wg = (warp - 2) >> 2;                  // query columns [32 wg, 32 wg + 32) of a block
     const int row = quarter * 32 + lane;             // key in the tile (S^T lane) / dh row (dQ^T lane)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    constexpr uint32_t kAct = 32 * kActWarps;
+    // The two warpgroups run independently: each has its own rab table, bucket
+    // sums, dQ staging half and named barrier (id 2 + wg, 128 threads).
+    const uint32_t bid = 2 + wg;
+    float* rabw = rab + wg * 64;
+    float* drabw = drab + wg * 64;
     const int d = P.A.d;
     uint32_t items_done = 0, g = 0;
     int cur_h = -1;
     const float inv_N = a.inv_N;
-    const int ti = threadIdx.x - 64;
+    const int tw = (threadIdx.x - 64) & 127;          // thread in the warpgroup
     bool fail = false;
     for (int it = blockIdx.x; it < total && !fail; it += gridDim.x) {
       const BItem item = P.w.items[it];
@@ -876,23 +924,29 @@ __global__ void __launch_bounds__(kBThreads, 1)
       const bool kvalid = jk < hlen;
       const long long tk = kvalid ? a.kv_ts[s0 + jk] : 0;
       if (item.h != cur_h) {
-        named_barrier(1, kAct);
-        if (cur_h >= 0 && ti < 64) {
-          float* dst = ti < 32 ? P.A.drab_pos : P.A.drab_time;
-          const int nb = ti < 32 ? a.P : a.Bt;
-          const int bi = ti & 31;
-          if (dst && bi < nb && drab[ti] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[ti] * inv_N);
+        named_barrier(bid, 128);
+        if (cur_h >= 0 && tw < 64) {
+          float* dst = tw < 32 ? P.A.drab_pos : P.A.drab_time;
+          const int nb = tw < 32 ? a.P : a.Bt;
+          const int bi = tw & 31;
+          if (dst && bi < nb && drabw[tw] != 0.f) atomicAdd(dst + cur_h * nb + bi, drabw[tw] * inv_N);
         }
-        if (ti < 32) {
-          rab[ti] = (a.rab_pos && ti < a.P) ? a.rab_pos[item.h * a.P + ti] : 0.f;
-          rab[32 + ti] = (a.rab_time && ti < a.Bt) ? a.rab_time[item.h * a.Bt + ti] : 0.f;
+        if (tw < 32) {
+          rabw[tw] = (a.rab_pos && tw < a.P) ? a.rab_pos[item.h * a.P + tw] : 0.f;
+          rabw[32 + tw] = (a.rab_time && tw < a.Bt) ? a.rab_time[item.h * a.Bt + tw] : 0.f;
         }
-        if (ti < 64) drab[ti] = 0.f;
-        named_barrier(1, kAct);
+        if (tw < 64) drabw[tw] = 0.f;
+        named_barrier(bid, 128);
         cur_h = item.h;
       }
-      if (named_barrier_any(1, kAct, *abort_flag != 0)) { fail = true; break; }
-      const float rp_far = rab[a.P - 1];
+      if (named_barrier_any(bid, 128, *abort_flag != 0)) { fail = true; break; }
+      if (kvalid) {
+        // the pre-activation lines the dK, dV epilogue reads at the item's end
+        const bf16* pr = static_cast<const bf16*>(P.A.pre) + (s0 + jk) * P.A.pre_stride + item.h * DH + wg * 64;
+        prefetch_l2(pr + d);
+        prefetch_l2(pr + 3 * d);
+      }
+      const float rp_far = rabw[a.P - 1];
       // dS sums per rab bucket of this key row: the last position bucket in a
       // register, the others and the time buckets run-length encoded (both
       // buckets are non-decreasing along the row's queries), flushed to
@@ -901,7 +955,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       int pb_cur = -1, tb_cur = -1;
       auto add_t = [&](int bkt, float v) {
         if (bkt != tb_cur) {
-          if (tb_cur >= 0) atomicAdd(&drab[32 + tb_cur], t_sum);
+          if (tb_cur >= 0) atomicAdd(&drabw[32 + tb_cur], t_sum);
           tb_cur = bkt;
           t_sum = 0.f;
         }
@@ -913,45 +967,50 @@ __global__ void __launch_bounds__(kBThreads, 1)
           return;
         }
         if (bkt != pb_cur) {
-          if (pb_cur >= 0) atomicAdd(&drab[pb_cur], p_sum);
+          if (pb_cur >= 0) atomicAdd(&drabw[pb_cur], p_sum);
           pb_cur = bkt;
           p_sum = 0.f;
         }
         p_sum += v;
       };
-      // drain dQ^T of block gd (query rows q0d ..): free its TMEM columns,
-      // transpose into the staging tile, one bulk reduce-add into dQ
-      auto drain = [&](uint32_t gd, int q0d) -> bool {
+      // drain this warpgroup's 32 queries of dQ^T of block gd (query rows
+      // q0d ..): free the TMEM columns, transpose into the warpgroup's staging
+      // half, one bulk reduce-add into dQ.  A failed wait only marks `fail`;
+      // the warpgroup stops together at its next barrier.
+      float* sdq = sDQ + wg * (32 * DH);
+      auto drain = [&](uint32_t gd, int q0d) {
         const uint32_t b = gd & 1;
         bool f = !mbar_wait(&dq_full[b], (gd >> 1) & 1, abort_flag, P.status);
-        if (ti == 0) bulk_wait_read0();             // the previous reduce has read the staging tile
-        if (named_barrier_any(1, kAct, f)) return false;
+        if (tw == 0) bulk_wait_read0();             // the previous reduce has read the staging half
+        if (named_barrier_any(bid, 128, f)) {
+          fail = true;
+          return;
+        }
         tc_fence_after();
         uint32_t r[32];
-        tmem_ld32(tS[b] + lane_off + wg * 32, r);
+        tmem_ld32(tS(b) + lane_off + wg * 32, r);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_free[b]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sDQ[(wg * 32 + i) * DH + row] = __uint_as_float(r[i]) * inv_N;
+        for (int i = 0; i < 32; ++i) sdq[i * DH + row] = __uint_as_float(r[i]) * inv_N;
         fence_proxy_async_smem();
-        named_barrier(1, kAct);
-        if (ti == 0) {
-          tma_reduce_add_2d(&tmdQ, sDQ, item.h * DH, (int32_t)(s0 + q0d));
+        named_barrier(bid, 128);
+        if (tw == 0) {
+          tma_reduce_add_2d(&tmdQ, sdq, item.h * DH, (int32_t)(s0 + q0d + wg * 32));
           bulk_commit();
         }
-        return true;
       };
 
       for (int m = 0; m < nqb; ++m) {
         const uint32_t gb = g + m, b = gb & 1;
         const int st = (int)(gb % kQStages);
         const int q0 = k0 + m * kQB;
-        fail = !mbar_wait(&st_full[b], (gb >> 1) & 1, abort_flag, P.status);
-        if (named_barrier_any(1, kAct, fail)) { fail = true; break; }
+        fail = !mbar_wait(&st_full[b], (gb >> 1) & 1, abort_flag, P.status) || fail;
+        if (named_barrier_any(bid, 128, fail)) { fail = true; break; }
         tc_fence_after();
-        const long long* qts = reinterpret_cast<const long long*>(sQD + st * C::QSTAGE + 2 * C::QTILE);
+        const long long* qts = reinterpret_cast<const long long*>(sTS + st * C::TS_BYTES);
         const int qf = q0 + wg * 32;                 // first query of this warpgroup's 32
         const bool full = kvalid && qf + 31 < n && jk <= qf;
         const bool far = min(qf, hlen) - jk >= a.P - 1;
@@ -962,8 +1021,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         const bool fast = __all_sync(0xffffffffu, full && far && nb <= 2);
         uint32_t sr[32], dr[32], pk[16], dk[16];
-        tmem_ld32(tS[b] + lane_off + wg * 32, sr);
-        tmem_ld32(tD[b] + lane_off + wg * 32, dr);
+        tmem_ld32(tS(b) + lane_off + wg * 32, sr);
+        tmem_ld32(tD(b) + lane_off + wg * 32, dr);
         tmem_ld_wait();
         if (fast) {
           const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)nb);
@@ -974,18 +1033,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
             if (k < nb) {
               const int bb = b_lo + 1 + k;
               // this half's queries (sorted) with t <= tk + 2^(bb-1) - 1
-              const long long tau = tk + (1LL << (bb - 1)) - 1;
-              const longlong2* q2 = reinterpret_cast<const longlong2*>(qts + wg * 32);
-              int cnt = 0;
-#pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const longlong2 v = q2[c];
-                cnt += (v.x <= tau) + (v.y <= tau);
-              }
-              p[k] = cnt;
-              hd[k] = 0.5f * (rab[32 + bb] - rab[32 + bb - 1]);
+              p[k] = count_le_32(qts + wg * 32, tk + (1LL << (bb - 1)) - 1);
+              hd[k] = 0.5f * (rabw[32 + bb] - rabw[32 + bb - 1]);
             }
-          const float hb = 0.5f * (rp_far + rab[32 + b_lo]);
+          const float hb = 0.5f * (rp_far + rabw[32 + b_lo]);
           float tot = 0.f, suf[2] = {0.f, 0.f};
           if (nbw == 0) bwd_chunk_fast<0>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
           else if (nbw == 1) bwd_chunk_fast<1>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
@@ -1012,7 +1063,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
               if (ok) {
                 const int bp = min(max(min(qpos, hlen) - jk, 0), a.P - 1);
                 const int bt = tb64(qts[col] - tk, a.Bt);
-                const float h = 0.5f * (__uint_as_float(sr[e + u]) + rab[bp] + rab[32 + bt]);
+                const float h = 0.5f * (__uint_as_float(sr[e + u]) + rabw[bp] + rabw[32 + bt]);
                 const float t = tanh_fast(h);
                 const float sg = fmaf(t, 0.5f, 0.5f);
                 pa = fmaf(h, t, h);
@@ -1027,8 +1078,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
             dk[e / 2] = pack_bf16(dv[0], dv[1]);
           }
         }
-        tmem_st16(tS[b] + lane_off + wg * 32, pk);
-        tmem_st16(tD[b] + lane_off + wg * 32, dk);
+        tmem_st16(tS(b) + lane_off + wg * 32, pk);
+        tmem_st16(tD(b) + lane_off + wg * 32, dk);
         uint8_t* dsb = sDS + b * C::DS_BYTES;
 #pragma unroll
         for (int g8 = 0; g8 < 4; ++g8) {
@@ -1040,21 +1091,21 @@ __global__ void __launch_bounds__(kBThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pds_full[b]);
-        if (m >= 1 && !drain(gb - 1, q0 - kQB)) { fail = true; break; }
+        if (m >= 1) drain(gb - 1, q0 - kQB);
       }
       if (fail) break;
-      if (nqb >= 1 && !drain(g + nqb - 1, k0 + (nqb - 1) * kQB)) { fail = true; break; }
+      if (nqb >= 1) drain(g + nqb - 1, k0 + (nqb - 1) * kQB);
       // flush this key row's bucket sums
-      if (tb_cur >= 0) atomicAdd(&drab[32 + tb_cur], t_sum);
-      if (pb_cur >= 0) atomicAdd(&drab[pb_cur], p_sum);
+      if (tb_cur >= 0) atomicAdd(&drabw[32 + tb_cur], t_sum);
+      if (pb_cur >= 0) atomicAdd(&drabw[pb_cur], p_sum);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) far_sum += __shfl_xor_sync(0xffffffffu, far_sum, o);
-      if (lane == 0 && far_sum != 0.f) atomicAdd(&drab[a.P - 1], far_sum);
+      if (lane == 0 && far_sum != 0.f) atomicAdd(&drabw[a.P - 1], far_sum);
       g += nqb;
       // this warpgroup's half of dK, dV (times 1/N and SiLU'(Pre)) into dPre
-      fail = !mbar_wait(dkv_full, items_done & 1, abort_flag, P.status);
+      fail = !mbar_wait(dkv_full, items_done & 1, abort_flag, P.status) || fail;
       ++items_done;
-      if (named_barrier_any(1, kAct, fail)) { fail = true; break; }
+      if (named_barrier_any(bid, 128, fail)) { fail = true; break; }
       tc_fence_after();
       const bf16* pre = static_cast<const bf16*>(P.A.pre);
       bf16* dpre = static_cast<bf16*>(P.A.dpre);
@@ -1096,14 +1147,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
       if (lane == 0) mbar_arrive(dkv_free);
     }
     // flush the last head's bucket sums
-    named_barrier(1, kAct);
-    if (cur_h >= 0 && ti < 64) {
-      float* dst = ti < 32 ? P.A.drab_pos : P.A.drab_time;
-      const int nb = ti < 32 ? a.P : a.Bt;
-      const int bi = ti & 31;
-      if (dst && bi < nb && drab[ti] != 0.f) atomicAdd(dst + cur_h * nb + bi, drab[ti] * inv_N);
+    named_barrier(bid, 128);
+    if (cur_h >= 0 && tw < 64) {
+      float* dst = tw < 32 ? P.A.drab_pos : P.A.drab_time;
+      const int nb = tw < 32 ? a.P : a.Bt;
+      const int bi = tw & 31;
+      if (dst && bi < nb && drabw[tw] != 0.f) atomicAdd(dst + cur_h * nb + bi, drabw[tw] * inv_N);
     }
-    if (ti == 0) bulk_wait0();
+    if (tw == 0) bulk_wait0();
   }
 
   tc_fence_before();
@@ -1167,8 +1218,8 @@ cudaError_t launch_bwd3(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaSt
             encode_tmap_2d(&tK, false, a.k, (uint64_t)d, (uint64_t)a.kv_rows, (uint64_t)a.kv_stride, 64, kT) &&
             encode_tmap_2d(&tV, false, a.v, (uint64_t)d, (uint64_t)a.kv_rows, (uint64_t)a.kv_stride, 64, kT) &&
             encode_tmap_2d(&tdO, false, A.dout, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)a.o_stride, 64, kQB);
-  CUtensorMap tdQ;  // fp32 [T][d] accumulator, dense 128 x 64 boxes, no swizzle
-  ok = ok && encode_tmap_2d(&tdQ, true, A.dq_acc, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)A.d, 128, kQB,
+  CUtensorMap tdQ;  // fp32 [T][d] accumulator, dense 128 x 32 boxes, no swizzle
+  ok = ok && encode_tmap_2d(&tdQ, true, A.dq_acc, (uint64_t)d, (uint64_t)a.q_rows, (uint64_t)A.d, 128, 32,
                             false);
   if (!ok) return cudaErrorInvalidValue;
   BSched w = bsched(ws);

@@ -336,10 +336,13 @@ int64_t hstu_launch_count(void);
 
 /* Device status word of this library on the current device: bit
  * HSTU_DEVICE_TIMEOUT is set when a kernel's bounded wait ran out (the kernel
- * then abandoned its work and exited cleanly; its outputs are not valid).
- * Copies the word to *host_out, synchronising `stream`; clears it when
- * `clear` is non-zero. */
+ * then abandoned its work and exited cleanly; its outputs are not valid);
+ * bit HSTU_DEVICE_SMEM_ALIGN when a kernel that packs its whole shared-memory
+ * budget found its dynamic shared memory not 1024-byte aligned (it exits at
+ * once; outputs not valid).  Copies the word to *host_out, synchronising
+ * `stream`; clears it when `clear` is non-zero. */
 #define HSTU_DEVICE_TIMEOUT 0x100u
+#define HSTU_DEVICE_SMEM_ALIGN 0x200u
 hstu_status hstu_device_status(uint32_t* host_out, int32_t clear, cudaStream_t stream);
 
 const char* hstu_status_string(hstu_status s);

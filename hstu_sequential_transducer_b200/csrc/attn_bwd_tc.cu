@@ -34,6 +34,8 @@
 // the per-bucket sums of dS: a total and one suffix sum per breakpoint.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -173,13 +175,13 @@ __device__ __forceinline__ int count_le_32(const long long* cts, long long tau) 
 // One 32-column chunk of the fast path: h = S/2 + bias/2 where columns
 // c >= p[k] add hd[k]; writes packed P and dS (unscaled) and accumulates the
 // total and the per-breakpoint suffix sums of dS.
-template <int NB>
+template <int NB, int E0 = 0, int NE = 32>
 __device__ __forceinline__ void bwd_chunk_fast(const uint32_t (&sr)[32], const uint32_t (&dr)[32],
                                                int c0, float hb, const int (&p)[2],
                                                const float (&hd)[2], uint32_t (&pk)[16],
                                                uint32_t (&dk)[16], float& tot, float (&suf)[2]) {
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
+  for (int e = E0; e < E0 + NE; e += 2) {
     float pa[2], ds[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -642,24 +644,26 @@ int sms();
 // ---------------------------------------------------------------------------
 // Pipelined backward for dh = 128: 64-query blocks
 // ---------------------------------------------------------------------------
-// With 64-query blocks two S^T/dP^T buffer pairs (4 x 64 TMEM columns) fit
-// next to the resident dV and dK accumulators (2 x 128), so the MMA thread
-// issues block g's S^T = K Q_g^T and dP^T = V dO_g^T before it waits for the
-// activation of block g-1, whose dV, dK and dQ^T MMAs then overlap the
-// activation of block g.  dQ^T_g = K^T dS_g (M = dh rows, 64 query columns)
-// goes into block g's S^T columns once dV has read P^T from them; the
-// activation warps drain it one block behind: each warpgroup transposes its
-// 32 queries into a dense 32 x 128 fp32 tile in shared memory and adds it to
-// the fp32 dQ accumulator with one TMA bulk reduce-add (rows past the
-// sequence end carry exact zeros).  Q/dO blocks come through a three-stage
-// ring, so that the loads of block g+1 are in flight while block g-1's dV and
-// dK still read their stage; the block times have a ring of their own.  This
-// packs the whole 227 KB budget, so the kernel relies on a 1024-byte aligned
+// A CTA owns one (key tile, head) item at a time and walks its query blocks
+// g = 0, 1, ... .  Per block the MMA thread computes S^T = K Q_g^T and
+// dP^T = V dO_g^T (128 keys x 64 queries, fp32 in TMEM); the activation warps
+// load both into registers, release the TMEM at once, and write P^T and dS
+// (bf16, [key][query] 128-byte swizzled tiles) to shared memory.  From there
+// the same tiles serve as the K-major A operand of dV += P^T dO and
+// dK += dS^T Q and as the MN-major B operand of dQ^T_g = K^T dS^T.  dQ^T has a
+// double buffer of its own in TMEM, so the next block's S^T, dP^T never wait
+// for the dQ drain: S^T(g+1) is issued as soon as block g's scores are in
+// registers, and the activation warps drain dQ^T(g-1) after finishing block g
+// (each warpgroup transposes its 32 queries into a dense fp32 tile in shared
+// memory and adds it to the fp32 dQ accumulator with one TMA bulk reduce-add;
+// rows past the sequence end carry exact zeros).  Q/dO blocks come through a
+// two-stage ring that the producer keeps prefetched into L2.  The layout packs
+// almost the whole 227 KB budget, so the kernel relies on a 1024-byte aligned
 // dynamic shared memory base (checked; it reports kStatusSmemAlign if not).
-// TMEM: S^T_0 [0,64) dP^T_0 [64,128) S^T_1 [128,192) dP^T_1 [192,256)
+// TMEM: S^T [0,64) dP^T [64,128) dQ^T_0 [128,192) dQ^T_1 [192,256)
 //       dV [256,384) dK [384,512)
 constexpr int kQB = 64;
-constexpr int kQStages = 3;
+constexpr int kQStages = 2;
 
 struct B3Cfg {
   static constexpr int DH = 128;
@@ -667,10 +671,10 @@ struct B3Cfg {
   static constexpr int QTILE = kQB * DH * 2;           // 64 queries x 128 bf16 = 16 KB
   static constexpr int QSTAGE = 2 * QTILE;             // Q, dO
   static constexpr int TS_BYTES = kQB * 8;             // one block's times
-  static constexpr int DS_BYTES = kT * kQB * 2;        // dS [key][query] for one block = 16 KB
+  static constexpr int PS_BYTES = kT * kQB * 2;        // P^T or dS [key][query] for one block = 16 KB
   static constexpr int DQ_BYTES = kQB * DH * 4;        // dQ staging, 2 x [32 queries][dh] fp32 = 32 KB
   static constexpr int BAR_BYTES = 1536;               // barriers, rab tables, TMEM slot
-  static constexpr int SMEM = 2 * KTILE + kQStages * QSTAGE + 2 * DS_BYTES + DQ_BYTES + kQStages * TS_BYTES +
+  static constexpr int SMEM = 2 * KTILE + kQStages * QSTAGE + 4 * PS_BYTES + DQ_BYTES + kQStages * TS_BYTES +
                               BAR_BYTES;
   static constexpr uint32_t IDESC_ST = idesc_bf16(128, kQB, false, false);   // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DKV = idesc_bf16(128, DH, false, true);    // P^T dO, dS^T Q
@@ -696,18 +700,21 @@ __global__ void __launch_bounds__(kBThreads, 1)
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::KTILE;
   uint8_t* sQD = sV + C::KTILE;                    // kQStages x (Q | dO)
-  uint8_t* sDS = sQD + kQStages * C::QSTAGE;        // 2 x dS
-  float* sDQ = reinterpret_cast<float*>(sDS + 2 * C::DS_BYTES);   // 2 x dQ staging [32][128]
-  uint8_t* sTS = sDS + 2 * C::DS_BYTES + C::DQ_BYTES;             // kQStages x times
+  uint8_t* sPT = sQD + kQStages * C::QSTAGE;        // 2 x P^T
+  uint8_t* sDS = sPT + 2 * C::PS_BYTES;             // 2 x dS
+  float* sDQ = reinterpret_cast<float*>(sDS + 2 * C::PS_BYTES);   // 2 x dQ staging [32][128]
+  uint8_t* sTS = sDS + 2 * C::PS_BYTES + C::DQ_BYTES;             // kQStages x times
   uint64_t* bars = reinterpret_cast<uint64_t*>(sTS + kQStages * C::TS_BYTES);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* qd_full = bars + 2;                     // [3]
-  uint64_t* qd_empty = bars + 5;                    // [3]
-  uint64_t* st_full = bars + 8;                     // [2]
-  uint64_t* pds_full = bars + 10;                   // [2] (8 warps)
-  uint64_t* dq_full = bars + 12;                    // [2]
-  uint64_t* a_free = bars + 14;                     // [2] (8 warps)
+  uint64_t* qd_full = bars + 2;                     // [2]
+  uint64_t* qd_empty = bars + 4;                    // [2]
+  uint64_t* st_full = bars + 6;                     // S^T, dP^T of the current block are in TMEM
+  uint64_t* s_free = bars + 7;                      // (8 warps) ... and have been read
+  uint64_t* pds_full = bars + 8;                    // [2] (8 warps) P^T, dS of a block are in smem
+  uint64_t* ps_free = bars + 10;                    // [2] the block's MMAs have read them
+  uint64_t* dq_full = bars + 12;                    // [2] dQ^T of a block is in TMEM
+  uint64_t* dq_free = bars + 14;                    // [2] (8 warps) ... and has been read
   uint64_t* dkv_full = bars + 16;
   uint64_t* dkv_free = bars + 17;                   // (8 warps)
   uint64_t* done_bar = bars + 18;
@@ -722,7 +729,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 19; ++i) {
-      const bool act = (i == 10 || i == 11 || i == 14 || i == 15 || i == 17);
+      const bool act = (i == 7 || i == 8 || i == 9 || i == 14 || i == 15 || i == 17);
       mbar_init(&bars[i], act ? kActWarps : 1);
     }
     *abort_flag = 0;
@@ -733,9 +740,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // S^T (then P^T, then dQ^T) of buffer b at columns 128 b, dP^T (then dS^T) at 128 b + 64
-  auto tS = [tmem](uint32_t b) { return tmem + b * 128u; };
-  auto tD = [tmem](uint32_t b) { return tmem + b * 128u + 64u; };
+  const uint32_t tS = tmem, tD = tmem + 64;
+  auto tQ = [tmem](uint32_t b) { return tmem + 128u + b * 64u; };
   const uint32_t tdV = tmem + 256, tdK = tmem + 384;
 
   if (warp == 0) {
@@ -838,52 +844,54 @@ __global__ void __launch_bounds__(kBThreads, 1)
         bool ok = true;
         for (int m = 0; m <= nqb && ok; ++m) {
           if (m < nqb) {
-            // block g + m: S^T, dP^T into buffer (g + m) & 1
-            const uint32_t gb = g + m, b = gb & 1;
+            // block g + m: S^T, dP^T once the previous block's are in registers
+            const uint32_t gb = g + m;
             const int st = (int)(gb % kQStages);
             if (!mbar_wait(&qd_full[st], (gb / kQStages) & 1, abort_flag, P.status)) { ok = false; break; }
-            if (gb >= 2 && !mbar_wait(&a_free[b], ((gb - 2) >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            if (gb >= 1 && !mbar_wait(s_free, (gb - 1) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t q_s = smem_u32(sQD + st * C::QSTAGE), do_s = q_s + C::QTILE;
 #pragma unroll
             for (int k = 0; k < DH / 16; ++k) {
               const uint32_t koff = (k / 4) * (kT * 128) + (k % 4) * 32;
               const uint32_t qoff = (k / 4) * (kQB * 128) + (k % 4) * 32;
-              mma_ss(tS(b), sdesc_kmajor(k_s + koff), sdesc_kmajor(q_s + qoff), C::IDESC_ST, k > 0);
+              mma_ss(tS, sdesc_kmajor(k_s + koff), sdesc_kmajor(q_s + qoff), C::IDESC_ST, k > 0);
             }
 #pragma unroll
             for (int k = 0; k < DH / 16; ++k) {
               const uint32_t koff = (k / 4) * (kT * 128) + (k % 4) * 32;
               const uint32_t qoff = (k / 4) * (kQB * 128) + (k % 4) * 32;
-              mma_ss(tD(b), sdesc_kmajor(v_s + koff), sdesc_kmajor(do_s + qoff), C::IDESC_ST, k > 0);
+              mma_ss(tD, sdesc_kmajor(v_s + koff), sdesc_kmajor(do_s + qoff), C::IDESC_ST, k > 0);
             }
-            mma_commit(&st_full[b]);
+            mma_commit(st_full);
           }
           if (m >= 1) {
-            // block g + m - 1: dV, dK accumulate; dQ^T into its S^T columns
+            // block g + m - 1: dV += P^T dO, dK += dS^T Q, dQ^T = K^T dS^T, all
+            // from the P^T and dS tiles the activation warps wrote to smem
             const uint32_t gp = g + m - 1, b = gp & 1;
             const int st = (int)(gp % kQStages);
             if (m == 1 && !mbar_wait(dkv_free, (items_done & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
             if (!mbar_wait(&pds_full[b], (gp >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            if (gp >= 2 && !mbar_wait(&dq_free[b], ((gp - 2) >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t q_s = smem_u32(sQD + st * C::QSTAGE), do_s = q_s + C::QTILE;
+            const uint32_t pt_s = smem_u32(sPT + b * C::PS_BYTES), ds_s = smem_u32(sDS + b * C::PS_BYTES);
             const uint32_t acc0 = m > 1 ? 1u : 0u;
-            // A operand halves: queries [0,32) at columns [0,16), [32,64) at [32,48)
 #pragma unroll
             for (int k = 0; k < kQB / 16; ++k)
-              mma_ts(tdV, tS(b) + (k / 2) * 32 + (k % 2) * 8, sdesc_mnmajor(do_s + k * 2048, kQB * 128),
-                     C::IDESC_DKV, (acc0 || k > 0) ? 1u : 0u);
+              mma_ss(tdV, sdesc_kmajor(pt_s + k * 32), sdesc_mnmajor(do_s + k * 2048, kQB * 128), C::IDESC_DKV,
+                     (acc0 || k > 0) ? 1u : 0u);
 #pragma unroll
             for (int k = 0; k < kQB / 16; ++k)
-              mma_ts(tdK, tD(b) + (k / 2) * 32 + (k % 2) * 8, sdesc_mnmajor(q_s + k * 2048, kQB * 128),
-                     C::IDESC_DKV, (acc0 || k > 0) ? 1u : 0u);
+              mma_ss(tdK, sdesc_kmajor(ds_s + k * 32), sdesc_mnmajor(q_s + k * 2048, kQB * 128), C::IDESC_DKV,
+                     (acc0 || k > 0) ? 1u : 0u);
             mma_commit(&qd_empty[st]);
-            const uint32_t ds_s = smem_u32(sDS + b * C::DS_BYTES);
 #pragma unroll
             for (int k = 0; k < kT / 16; ++k)
-              mma_ss(tS(b), sdesc_mnmajor(k_s + k * 2048, kT * 128), sdesc_mnmajor(ds_s + k * 2048, kT * 128),
+              mma_ss(tQ(b), sdesc_mnmajor(k_s + k * 2048, kT * 128), sdesc_mnmajor(ds_s + k * 2048, kT * 128),
                      C::IDESC_DQT, k > 0 ? 1u : 0u);
             mma_commit(&dq_full[b]);
+            mma_commit(&ps_free[b]);
           }
         }
         if (!ok) break;
@@ -974,9 +982,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
         p_sum += v;
       };
       // drain this warpgroup's 32 queries of dQ^T of block gd (query rows
-      // q0d ..): free the TMEM columns, transpose into the warpgroup's staging
-      // half, one bulk reduce-add into dQ.  A failed wait only marks `fail`;
-      // the warpgroup stops together at its next barrier.
+      // q0d ..): read its TMEM buffer and release it, transpose into the
+      // warpgroup's staging half, one bulk reduce-add into dQ.  A failed wait
+      // only marks `fail`; the warpgroup stops together at its next barrier.
       float* sdq = sDQ + wg * (32 * DH);
       auto drain = [&](uint32_t gd, int q0d) {
         const uint32_t b = gd & 1;
@@ -988,11 +996,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         tc_fence_after();
         uint32_t r[32];
-        tmem_ld32(tS(b) + lane_off + wg * 32, r);
+        tmem_ld32(tQ(b) + lane_off + wg * 32, r);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_free[b]);
+        if (lane == 0) mbar_arrive(&dq_free[b]);
 #pragma unroll
         for (int i = 0; i < 32; ++i) sdq[i * DH + row] = __uint_as_float(r[i]) * inv_N;
         fence_proxy_async_smem();
@@ -1007,9 +1015,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const uint32_t gb = g + m, b = gb & 1;
         const int st = (int)(gb % kQStages);
         const int q0 = k0 + m * kQB;
-        fail = !mbar_wait(&st_full[b], (gb >> 1) & 1, abort_flag, P.status) || fail;
+        fail = !mbar_wait(st_full, gb & 1, abort_flag, P.status) || fail;
         if (named_barrier_any(bid, 128, fail)) { fail = true; break; }
         tc_fence_after();
+        // S^T, dP^T loads in flight while the path is chosen
+        uint32_t sr[32], dr[32], pk[16], dk[16];
+        tmem_ld32(tS + lane_off + wg * 32, sr);
+        tmem_ld32(tD + lane_off + wg * 32, dr);
         const long long* qts = reinterpret_cast<const long long*>(sTS + st * C::TS_BYTES);
         const int qf = q0 + wg * 32;                 // first query of this warpgroup's 32
         const bool full = kvalid && qf + 31 < n && jk <= qf;
@@ -1020,14 +1032,16 @@ __global__ void __launch_bounds__(kBThreads, 1)
           nb = tb64(qts[wg * 32 + 31] - tk, a.Bt) - b_lo;
         }
         const bool fast = __all_sync(0xffffffffu, full && far && nb <= 2);
-        uint32_t sr[32], dr[32], pk[16], dk[16];
-        tmem_ld32(tS(b) + lane_off + wg * 32, sr);
-        tmem_ld32(tD(b) + lane_off + wg * 32, dr);
         tmem_ld_wait();
+        // the scores are in registers: the next block's may overwrite them
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        // fast path: columns c >= p[k] add hd[k] to the half-bias hb
+        int p[2] = {32, 32}, nbw = 0;
+        float hd[2] = {0.f, 0.f}, hb = 0.f, tot = 0.f, suf[2] = {0.f, 0.f};
         if (fast) {
-          const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)nb);
-          int p[2] = {32, 32};
-          float hd[2] = {0.f, 0.f};
+          nbw = __reduce_max_sync(0xffffffffu, (unsigned)nb);
 #pragma unroll
           for (int k = 0; k < 2; ++k)
             if (k < nb) {
@@ -1036,23 +1050,20 @@ __global__ void __launch_bounds__(kBThreads, 1)
               p[k] = count_le_32(qts + wg * 32, tk + (1LL << (bb - 1)) - 1);
               hd[k] = 0.5f * (rabw[32 + bb] - rabw[32 + bb - 1]);
             }
-          const float hb = 0.5f * (rp_far + rabw[32 + b_lo]);
-          float tot = 0.f, suf[2] = {0.f, 0.f};
-          if (nbw == 0) bwd_chunk_fast<0>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
-          else if (nbw == 1) bwd_chunk_fast<1>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
-          else bwd_chunk_fast<2>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
-          far_sum += tot;
-          float below = tot;
+          hb = 0.5f * (rp_far + rabw[32 + b_lo]);
+        }
+        // columns [E0, E0 + 16) of this warp's 32 (two halves keep the
+        // unrolled code and its register ranges small)
+        auto half = [&](auto e0c) {
+          constexpr int E0 = decltype(e0c)::value;
+          if (fast) {
+            if (nbw == 0) bwd_chunk_fast<0, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
+            else if (nbw == 1) bwd_chunk_fast<1, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
+            else bwd_chunk_fast<2, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
+            return;
+          }
 #pragma unroll
-          for (int k = 0; k < 2; ++k)
-            if (k < nb) {
-              add_t(b_lo + k, below - suf[k]);
-              below = suf[k];
-            }
-          add_t(b_lo + nb, below);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
+          for (int e = E0; e < E0 + 16; e += 2) {
             float pv[2], dv[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
@@ -1077,20 +1088,34 @@ __global__ void __launch_bounds__(kBThreads, 1)
             pk[e / 2] = pack_bf16(pv[0], pv[1]);
             dk[e / 2] = pack_bf16(dv[0], dv[1]);
           }
+        };
+        half(std::integral_constant<int, 0>{});
+        half(std::integral_constant<int, 16>{});
+        if (fast) {
+          far_sum += tot;
+          float below = tot;
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+            if (k < nb) {
+              add_t(b_lo + k, below - suf[k]);
+              below = suf[k];
+            }
+          add_t(b_lo + nb, below);
         }
-        tmem_st16(tS(b) + lane_off + wg * 32, pk);
-        tmem_st16(tD(b) + lane_off + wg * 32, dk);
-        uint8_t* dsb = sDS + b * C::DS_BYTES;
+        // P^T and dS into this block's tiles once block gb-2's MMAs have read them
+        if (gb >= 2) fail = !mbar_wait(&ps_free[b], ((gb - 2) >> 1) & 1, abort_flag, P.status) || fail;
+        uint8_t* ptb = sPT + b * C::PS_BYTES;
+        uint8_t* dsb = sDS + b * C::PS_BYTES;
 #pragma unroll
         for (int g8 = 0; g8 < 4; ++g8) {
-          const uint4 v = make_uint4(dk[4 * g8], dk[4 * g8 + 1], dk[4 * g8 + 2], dk[4 * g8 + 3]);
-          *reinterpret_cast<uint4*>(dsb + mn_off(row, wg * 32 + g8 * 8, kT * 128)) = v;
+          const uint32_t off = mn_off(row, wg * 32 + g8 * 8, kT * 128);
+          *reinterpret_cast<uint4*>(ptb + off) = make_uint4(pk[4 * g8], pk[4 * g8 + 1], pk[4 * g8 + 2], pk[4 * g8 + 3]);
+          *reinterpret_cast<uint4*>(dsb + off) = make_uint4(dk[4 * g8], dk[4 * g8 + 1], dk[4 * g8 + 2], dk[4 * g8 + 3]);
         }
-        tmem_st_wait();
         fence_proxy_async_smem();
-        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pds_full[b]);
+        // the previous block's dQ^T (its MMAs ran while this block was computed)
         if (m >= 1) drain(gb - 1, q0 - kQB);
       }
       if (fail) break;

@@ -10,14 +10,18 @@
 // Work items are (sequence, head, 128-row query tile), ordered longest-first
 // by a device-side counting sort (attn_sched) and dealt round-robin to one
 // persistent CTA per SM.  Per CTA:
-//   warp 0      TMA producer: Q tile once per item; K and V tiles (128 keys) and
-//               the keys' timestamps into a ring of stages
+//   warp 0      K producer: the Q tile once per item; K tiles (128 keys) with
+//               the keys' timestamps into a three-stage ring, freed as soon as
+//               S = Q K^T has read the tile
+//   warp 10     V producer: V tiles into a two-stage ring, freed by O += P V
 //   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S
 //               buffers; O += P V with P read from TMEM (A operand in TMEM)
 //   warps 2..9  two warpgroups, one query row per thread, each taking half of
 //               the 128 key columns: S from TMEM, bucketed rab bias, mask,
 //               SiLU, P (bf16) into a TMEM P buffer; at the end of an item,
 //               half of O each, times 1/N plus the candidates' self term
+// Both producers read timestamps ahead of their waits and keep the next
+// tiles prefetched into L2, so the rings refill at L2 latency.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O [256,384), P0 [384,448),
 // P1 [448,512).  A commit arrives only when every earlier MMA of the thread
 // is complete, so once S_{j+2} is signalled the PV of tile j has read P_j.
@@ -162,19 +166,19 @@ template <int DH>
 struct FwdCfg {
   static constexpr int BOXES = DH / 64;                 // 64-column boxes per tile row
   static constexpr int TILE_BYTES = kTile * DH * 2;     // one 128 x DH bf16 tile
-  static constexpr int STAGES = 2;
-  static constexpr int KV_BYTES = 2 * TILE_BYTES;       // K and V
-  static constexpr int TS_BYTES = kTile * 8;            // key timestamps
-  static constexpr int STAGE_BYTES = KV_BYTES + TS_BYTES;
-  static constexpr int SMEM_USED = 1024 + TILE_BYTES + STAGES * STAGE_BYTES + 1024;
+  static constexpr int K_STAGES = 3;                    // K tiles (and their timestamps)
+  static constexpr int V_STAGES = 2;                    // V tiles
+  static constexpr int TS_BYTES = kTile * 8;            // key timestamps of one K stage
+  static constexpr int SMEM_USED = 1024 + TILE_BYTES * (1 + K_STAGES + V_STAGES) + K_STAGES * TS_BYTES + 1024;
   // at least half of the SM's shared memory, so that one CTA (and its 512
   // TMEM columns) is resident per SM
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr uint32_t IDESC_S = idesc_bf16(128, kTile, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16(128, DH, false, true);
   static constexpr uint32_t TMEM_COLS = 512;            // S0, S1, O, P0, P1
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;                   // 11 warps (the V producer is warp 10)
   static constexpr int ACT_WARPS = 8;
+  static constexpr int PREFETCH = 4;                    // key tiles kept prefetched into L2
 };
 
 struct FwdParams {
@@ -227,20 +231,25 @@ __device__ __forceinline__ void act_chunk_fast(const uint32_t (&s)[32], int c0, 
 }
 
 template <int DH>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const FwdParams P) {
   using C = FwdCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sStage = sQ + C::TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + C::STAGES * C::STAGE_BYTES);
+  uint8_t* sK = sQ + C::TILE_BYTES;                      // K_STAGES tiles
+  uint8_t* sV = sK + C::K_STAGES * C::TILE_BYTES;        // V_STAGES tiles
+  uint8_t* sTS = sV + C::V_STAGES * C::TILE_BYTES;       // K_STAGES x timestamps
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sTS + C::K_STAGES * C::TS_BYTES);
   uint64_t* q_full = bars;                   // 1
   uint64_t* q_empty = bars + 1;              // 1
-  uint64_t* kv_full = bars + 2;              // STAGES
-  uint64_t* kv_empty = kv_full + C::STAGES;  // STAGES
-  uint64_t* s_full = kv_empty + C::STAGES;   // 2
+  uint64_t* k_full = bars + 2;               // K_STAGES
+  uint64_t* k_empty = k_full + C::K_STAGES;  // K_STAGES: S has read the K tile
+  uint64_t* ts_free = k_empty + C::K_STAGES; // K_STAGES (8 warps): the tile's timestamps are read
+  uint64_t* v_full = ts_free + C::K_STAGES;  // V_STAGES
+  uint64_t* v_empty = v_full + C::V_STAGES;  // V_STAGES
+  uint64_t* s_full = v_empty + C::V_STAGES;  // 2
   uint64_t* p_full = s_full + 2;             // 2
   uint64_t* o_full = p_full + 2;             // 1
   uint64_t* o_free = o_full + 1;             // 1
@@ -256,9 +265,14 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < C::K_STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&ts_free[s], C::ACT_WARPS);
+    }
+    for (int s = 0; s < C::V_STAGES; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -275,15 +289,16 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS[2] = {tmem, tmem + 128};
+  // S buffer b at columns [128 b, 128 b + 128), O at [256, 384), P buffer b at [384 + 64 b, ...)
+  auto tS = [tmem](uint32_t b) { return tmem + b * 128u; };
   const uint32_t tO = tmem + 256;
-  const uint32_t tP[2] = {tmem + 384, tmem + 448};
+  auto tP = [tmem](uint32_t b) { return tmem + 384u + b * 64u; };
 
   // Every role walks the same item sequence and numbers the key tiles it
-  // meets with one running counter n: K/V stage n % STAGES (parity
-  // (n / STAGES) & 1) and S/P buffer n & 1 (parity (n >> 1) & 1).
+  // meets with one running counter n: K stage n % K_STAGES (parity
+  // (n / K_STAGES) & 1), V stage n % V_STAGES, S/P buffer n & 1.
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ K producer
     uint32_t n = 0, items_done = 0;
     uint32_t issued = 0, issued_par = 0;
     bool q_issued = false;
@@ -296,6 +311,18 @@ __global__ void __launch_bounds__(320, 1)
       const int kend = item_kend(g, item.qt);
       const int nk = (kend + kTile - 1) / kTile;
       if (nk == 0) continue;
+      // L2 prefetch of key tile jp: K rows and their timestamps
+      auto prefetch = [&](int jp) {
+        if (jp >= nk) return;
+        const int kp = jp * kTile;
+        if (lane < C::BOXES) {
+          tma_prefetch_2d(&tmK, item.h * DH + 64 * lane, (int32_t)(g.ks + kp));
+        } else if (lane >= 8 && lane < 16) {
+          const int r = kp + (lane - 8) * 16;          // 16 times per 128-byte line
+          if (r < kend) prefetch_l2(a.kv_ts + g.ks + r);
+        }
+      };
+      for (int jp = 0; jp < C::PREFETCH; ++jp) prefetch(jp);
       bool ok = true;
       if (lane == 0) ok = mbar_wait(q_empty, (items_done & 1) ^ 1, abort_flag, P.status);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -310,30 +337,34 @@ __global__ void __launch_bounds__(320, 1)
       }
       ++items_done;
       for (int j = 0; j < nk; ++j, ++n) {
-        const int stage = (int)(n % C::STAGES);
-        const uint32_t par = (n / C::STAGES) & 1;
-        if (lane == 0) ok = mbar_wait(&kv_empty[stage], par ^ 1, abort_flag, P.status);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        uint8_t* st = sStage + stage * C::STAGE_BYTES;
-        long long* kts = reinterpret_cast<long long*>(st + C::KV_BYTES);
+        const int stage = (int)(n % C::K_STAGES);
+        const uint32_t par = (n / C::K_STAGES) & 1;
         const int k0 = j * kTile;
+        prefetch(j + C::PREFETCH);
+        // the tile's times, read while the stage is still in use; past the
+        // visible keys a large sentinel keeps the staged times sorted
+        long long tk[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int c = lane + 32 * q;
-          // past the visible keys: a large sentinel keeps the staged times sorted
-          kts[c] = (k0 + c < kend) ? a.kv_ts[g.ks + k0 + c] : (1LL << 62);
+          tk[q] = (k0 + c < kend) ? a.kv_ts[g.ks + k0 + c] : (1LL << 62);
         }
+        if (lane == 0) {
+          ok = mbar_wait(&k_empty[stage], par ^ 1, abort_flag, P.status);
+          ok = ok && mbar_wait(&ts_free[stage], par ^ 1, abort_flag, P.status);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        long long* kts = reinterpret_cast<long long*>(sTS + stage * C::TS_BYTES);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) kts[lane + 32 * q] = tk[q];
         __syncwarp();
         if (lane == 0) {
-          mbar_expect_tx(&kv_full[stage], C::KV_BYTES);
+          mbar_expect_tx(&k_full[stage], C::TILE_BYTES);
 #pragma unroll
-          for (int x = 0; x < C::BOXES; ++x) {
-            tma_load_2d(st + x * (kTile * 128), &tmK, &kv_full[stage], item.h * DH + 64 * x,
-                        (int32_t)(g.ks + k0));
-            tma_load_2d(st + C::TILE_BYTES + x * (kTile * 128), &tmV, &kv_full[stage],
+          for (int x = 0; x < C::BOXES; ++x)
+            tma_load_2d(sK + stage * C::TILE_BYTES + x * (kTile * 128), &tmK, &k_full[stage],
                         item.h * DH + 64 * x, (int32_t)(g.ks + k0));
-          }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (par << stage);
         }
@@ -342,9 +373,48 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (lane == 0) {
       volatile int never = 0;
-      for (int s2 = 0; s2 < C::STAGES; ++s2)
-        if (issued & (1u << s2)) mbar_wait(&kv_full[s2], (issued_par >> s2) & 1u, &never, P.status);
+      for (int s2 = 0; s2 < C::K_STAGES; ++s2)
+        if (issued & (1u << s2)) mbar_wait(&k_full[s2], (issued_par >> s2) & 1u, &never, P.status);
       if (q_issued) mbar_wait(q_full, q_par, &never, P.status);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ V producer
+    uint32_t n = 0, issued = 0, issued_par = 0;
+    for (int it = blockIdx.x; it < total; it += gridDim.x) {
+      if (*abort_flag) break;
+      const AttnItem item = P.w.items[it];
+      const SeqGeom g = seq_geom(a, item.b);
+      const int kend = item_kend(g, item.qt);
+      const int nk = (kend + kTile - 1) / kTile;
+      if (nk == 0) continue;
+      auto prefetch = [&](int jp) {
+        if (jp < nk && lane < C::BOXES) tma_prefetch_2d(&tmV, item.h * DH + 64 * lane, (int32_t)(g.ks + jp * kTile));
+      };
+      for (int jp = 0; jp < C::PREFETCH; ++jp) prefetch(jp);
+      bool ok = true;
+      for (int j = 0; j < nk; ++j, ++n) {
+        const int stage = (int)(n % C::V_STAGES);
+        const uint32_t par = (n / C::V_STAGES) & 1;
+        prefetch(j + C::PREFETCH);
+        if (lane == 0) ok = mbar_wait(&v_empty[stage], par ^ 1, abort_flag, P.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(&v_full[stage], C::TILE_BYTES);
+#pragma unroll
+          for (int x = 0; x < C::BOXES; ++x)
+            tma_load_2d(sV + stage * C::TILE_BYTES + x * (kTile * 128), &tmV, &v_full[stage],
+                        item.h * DH + 64 * x, (int32_t)(g.ks + j * kTile));
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (par << stage);
+        }
+      }
+      if (!ok) break;
+    }
+    if (lane == 0) {
+      volatile int never = 0;
+      for (int s2 = 0; s2 < C::V_STAGES; ++s2)
+        if (issued & (1u << s2)) mbar_wait(&v_full[s2], (issued_par >> s2) & 1u, &never, P.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -365,31 +435,33 @@ __global__ void __launch_bounds__(320, 1)
           if (j < nk) {
             // S_j = Q K_j^T into buffer (n + j) & 1
             const uint32_t nj = n + j;
-            const int stage = (int)(nj % C::STAGES);
-            if (!mbar_wait(&kv_full[stage], (nj / C::STAGES) & 1, abort_flag, P.status)) { ok = false; break; }
+            const int stage = (int)(nj % C::K_STAGES);
+            if (!mbar_wait(&k_full[stage], (nj / C::K_STAGES) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t k0s = smem_u32(sStage + stage * C::STAGE_BYTES);
+            const uint32_t k0s = smem_u32(sK + stage * C::TILE_BYTES);
 #pragma unroll
             for (int k = 0; k < DH / 16; ++k) {
               const uint32_t off = (k / 4) * (kTile * 128) + (k % 4) * 32;
-              mma_ss(tS[nj & 1], sdesc_kmajor(q0 + off), sdesc_kmajor(k0s + off), C::IDESC_S, k > 0);
+              mma_ss(tS(nj & 1), sdesc_kmajor(q0 + off), sdesc_kmajor(k0s + off), C::IDESC_S, k > 0);
             }
             mma_commit(&s_full[nj & 1]);
+            mma_commit(&k_empty[stage]);
             if (j == nk - 1) mma_commit(q_empty);
           }
           if (j >= 1) {
             // O += P_{j-1} V_{j-1}
             const uint32_t np = n + j - 1;
             if (j == 1 && !mbar_wait(o_free, (items_done & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
+            const int pst = (int)(np % C::V_STAGES);
+            if (!mbar_wait(&v_full[pst], (np / C::V_STAGES) & 1, abort_flag, P.status)) { ok = false; break; }
             if (!mbar_wait(&p_full[np & 1], (np >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
-            const int pst = (int)(np % C::STAGES);
-            const uint32_t v0 = smem_u32(sStage + pst * C::STAGE_BYTES) + C::TILE_BYTES;
+            const uint32_t v0 = smem_u32(sV + pst * C::TILE_BYTES);
 #pragma unroll
             for (int k = 0; k < kTile / 16; ++k)
-              mma_ts(tO, tP[np & 1] + k * 8, sdesc_mnmajor(v0 + k * 2048, kTile * 128), C::IDESC_O,
+              mma_ts(tO, tP(np & 1) + k * 8, sdesc_mnmajor(v0 + k * 2048, kTile * 128), C::IDESC_O,
                      (j > 1 || k > 0) ? 1u : 0u);
-            mma_commit(&kv_empty[pst]);
+            mma_commit(&v_empty[pst]);
           }
         }
         if (!ok) break;
@@ -401,7 +473,7 @@ __global__ void __launch_bounds__(320, 1)
       volatile int never = 0;
       mbar_wait(done_bar, 0, &never, P.status);
     }
-  } else {
+  } else if (warp < 2 + C::ACT_WARPS) {
     // ------------------------------------------------------------ activation + epilogue
     const int quarter = warp & 3;
     const int wg = (warp - 2) >> 2;                 // warpgroup: key columns [64 wg, 64 wg + 64)
@@ -442,8 +514,8 @@ __global__ void __launch_bounds__(320, 1)
         fail = !mbar_wait(&s_full[buf], par, abort_flag, P.status);
         if (named_barrier_any(1, kActThreads, fail)) { fail = true; break; }
         tc_fence_after();
-        const int kst = (int)(nj % C::STAGES);
-        const long long* kts = reinterpret_cast<const long long*>(sStage + kst * C::STAGE_BYTES + C::KV_BYTES);
+        const int kst = (int)(nj % C::K_STAGES);
+        const long long* kts = reinterpret_cast<const long long*>(sTS + kst * C::TS_BYTES);
         const int k0 = j * kTile;
         // fast path: every key of the tile visible, last position bucket,
         // at most two time-bucket breakpoints along the row
@@ -456,8 +528,8 @@ __global__ void __launch_bounds__(320, 1)
           nb = b_hi - b_lo;
         }
         const bool fast = __all_sync(0xffffffffu, rvalid && full_tile && far && nb <= 2);
-        const uint32_t sbuf = tS[buf] + lane_off + wg * 64;
-        const uint32_t pbuf = tP[buf] + lane_off + wg * 32;
+        const uint32_t sbuf = tS(buf) + lane_off + wg * 64;
+        const uint32_t pbuf = tP(buf) + lane_off + wg * 32;
         if (fast) {
           const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)nb);
           int p[2] = {0, 0};
@@ -507,7 +579,10 @@ __global__ void __launch_bounds__(320, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[buf]);
+        if (lane == 0) {
+          mbar_arrive(&p_full[buf]);
+          mbar_arrive(&ts_free[kst]);
+        }
       }
       if (fail) break;
       n += nk;

@@ -16,10 +16,13 @@
 //   warp 10     V producer: V tiles into a two-stage ring, freed by O += P V
 //   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S
 //               buffers; O += P V with P read from TMEM (A operand in TMEM)
-//   warps 2..9  two warpgroups, one query row per thread, each taking half of
-//               the 128 key columns: S from TMEM, bucketed rab bias, mask,
-//               SiLU, P (bf16) into a TMEM P buffer; at the end of an item,
-//               half of O each, times 1/N plus the candidates' self term
+//   warps 2..9  two warpgroups, one query row per thread; warpgroup b takes
+//               the key tiles of S/P buffer b (every other tile, all 128
+//               columns), so one warpgroup's waits and bucket searches
+//               overlap the other's SiLU work: S from TMEM, bucketed rab
+//               bias, mask, SiLU, P (bf16) into its TMEM P buffer; at the
+//               end of an item, half of O each, times 1/N plus the
+//               candidates' self term
 // Both producers read timestamps ahead of their waits and keep the next
 // tiles prefetched into L2, so the rings refill at L2 latency.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O [256,384), P0 [384,448),
@@ -230,6 +233,21 @@ __device__ __forceinline__ void act_chunk_fast(const uint32_t (&s)[32], int c0, 
   }
 }
 
+// The fast path over a whole 128-column tile, 32 columns at a time (the
+// other warpgroup's work covers the TMEM load latency).
+template <int NB>
+__device__ __forceinline__ void act_tile_fast(uint32_t sbuf, uint32_t pbuf, float hb, const int (&p)[2],
+                                              const float (&hd)[2]) {
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    uint32_t sv[32], pk[16];
+    tmem_ld32(sbuf + c * 32, sv);
+    tmem_ld_wait();
+    act_chunk_fast<NB>(sv, c * 32, hb, p, hd, pk);
+    tmem_st16(pbuf + c * 16, pk);
+  }
+}
+
 template <int DH>
 __global__ void __launch_bounds__(352, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -254,8 +272,8 @@ __global__ void __launch_bounds__(352, 1)
   uint64_t* o_full = p_full + 2;             // 1
   uint64_t* o_free = o_full + 1;             // 1
   uint64_t* done_bar = o_free + 1;           // 1
-  float* rab = reinterpret_cast<float*>(done_bar + 1);   // [2][32] of the current head
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rab + 64);
+  float* rab_all = reinterpret_cast<float*>(done_bar + 1);   // per warpgroup [2][32] of its head
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rab_all + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const AttnArgs& a = P.a;
@@ -268,7 +286,7 @@ __global__ void __launch_bounds__(352, 1)
     for (int s = 0; s < C::K_STAGES; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
-      mbar_init(&ts_free[s], C::ACT_WARPS);
+      mbar_init(&ts_free[s], C::ACT_WARPS / 2);      // the warpgroup that took the tile
     }
     for (int s = 0; s < C::V_STAGES; ++s) {
       mbar_init(&v_full[s], 1);
@@ -276,7 +294,7 @@ __global__ void __launch_bounds__(352, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], C::ACT_WARPS);
+      mbar_init(&p_full[i], C::ACT_WARPS / 2);       // the warpgroup of buffer i
     }
     mbar_init(o_full, 1);
     mbar_init(o_free, C::ACT_WARPS);
@@ -476,10 +494,11 @@ __global__ void __launch_bounds__(352, 1)
   } else if (warp < 2 + C::ACT_WARPS) {
     // ------------------------------------------------------------ activation + epilogue
     const int quarter = warp & 3;
-    const int wg = (warp - 2) >> 2;                 // warpgroup: key columns [64 wg, 64 wg + 64)
+    const int wg = (warp - 2) >> 2;                 // takes the tiles of buffer wg; O columns [DH/2 wg, ...)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    constexpr uint32_t kActThreads = 32 * C::ACT_WARPS;
+    const uint32_t bid = 2 + wg;                    // this warpgroup's named barrier (128 threads)
+    float* rab = rab_all + wg * 64;
     uint32_t n = 0, items_done = 0;
     int cur_h = -1;
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
@@ -495,24 +514,24 @@ __global__ void __launch_bounds__(352, 1)
       const bool cand = qpos >= g.hlen;
       const long long tq = rvalid ? a.q_ts[g.qs + r0 + row] : 0;
       if (item.h != cur_h) {
-        named_barrier(1, kActThreads);
-        if (threadIdx.x - 64 < 32) {
-          const int t = threadIdx.x - 64;
+        named_barrier(bid, 128);
+        const int t = (threadIdx.x - 64) & 127;
+        if (t < 32) {
           rab[t] = (a.rab_pos && t < a.P) ? a.rab_pos[item.h * a.P + t] : 0.f;
           rab[32 + t] = (a.rab_time && t < a.Bt) ? a.rab_time[item.h * a.Bt + t] : 0.f;
         }
-        named_barrier(1, kActThreads);
+        named_barrier(bid, 128);
         cur_h = item.h;
       }
       bool stop = *abort_flag != 0;
-      if (named_barrier_any(1, kActThreads, stop)) break;
+      if (named_barrier_any(bid, 128, stop)) break;
       bool fail = false;
       const float rp_far = rab[a.P - 1];
-      for (int j = 0; j < nk; ++j) {
+      for (int j = (int)((n + wg) & 1); j < nk; j += 2) {   // the tiles of buffer wg
         const uint32_t nj = n + j;
         const uint32_t buf = nj & 1, par = (nj >> 1) & 1;
         fail = !mbar_wait(&s_full[buf], par, abort_flag, P.status);
-        if (named_barrier_any(1, kActThreads, fail)) { fail = true; break; }
+        if (named_barrier_any(bid, 128, fail)) { fail = true; break; }
         tc_fence_after();
         const int kst = (int)(nj % C::K_STAGES);
         const long long* kts = reinterpret_cast<const long long*>(sTS + kst * C::TS_BYTES);
@@ -528,8 +547,8 @@ __global__ void __launch_bounds__(352, 1)
           nb = b_hi - b_lo;
         }
         const bool fast = __all_sync(0xffffffffu, rvalid && full_tile && far && nb <= 2);
-        const uint32_t sbuf = tS(buf) + lane_off + wg * 64;
-        const uint32_t pbuf = tP(buf) + lane_off + wg * 32;
+        const uint32_t sbuf = tS(buf) + lane_off;
+        const uint32_t pbuf = tP(buf) + lane_off;
         if (fast) {
           const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)nb);
           int p[2] = {0, 0};
@@ -538,23 +557,16 @@ __global__ void __launch_bounds__(352, 1)
           for (int k = 0; k < 2; ++k)
             if (k < nb) {
               const int b = b_lo + 1 + k;
-              p[k] = count_le128(kts, tq - (1LL << (b - 1))) - wg * 64;
+              p[k] = count_le128(kts, tq - (1LL << (b - 1)));
               hd[k] = 0.5f * (rab[32 + b] - rab[32 + b - 1]);
             }
           const float hb = 0.5f * (rp_far + rab[32 + b_lo]);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t sv[32], pk[16];
-            tmem_ld32(sbuf + c * 32, sv);
-            tmem_ld_wait();
-            if (nbw == 0) act_chunk_fast<0>(sv, c * 32, hb, p, hd, pk);
-            else if (nbw == 1) act_chunk_fast<1>(sv, c * 32, hb, p, hd, pk);
-            else act_chunk_fast<2>(sv, c * 32, hb, p, hd, pk);
-            tmem_st16(pbuf + c * 16, pk);
-          }
+          if (nbw == 0) act_tile_fast<0>(sbuf, pbuf, hb, p, hd);
+          else if (nbw == 1) act_tile_fast<1>(sbuf, pbuf, hb, p, hd);
+          else act_tile_fast<2>(sbuf, pbuf, hb, p, hd);
         } else {
 #pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < 4; ++c) {
             uint32_t sv[32], pk[16];
             tmem_ld32(sbuf + c * 32, sv);
             tmem_ld_wait();
@@ -563,7 +575,7 @@ __global__ void __launch_bounds__(352, 1)
               float y[2];
 #pragma unroll
               for (int u = 0; u < 2; ++u) {
-                const int col = wg * 64 + c * 32 + e + u;
+                const int col = c * 32 + e + u;
                 const int jk = k0 + col;
                 const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
                 const int bp = min(max(qp_clamped - jk, 0), a.P - 1);
@@ -612,7 +624,7 @@ __global__ void __launch_bounds__(352, 1)
       if (nk > 0) {
         fail = !mbar_wait(o_full, items_done & 1, abort_flag, P.status);
         ++items_done;
-        if (named_barrier_any(1, kActThreads, fail)) break;
+        if (named_barrier_any(bid, 128, fail)) break;
         tc_fence_after();
       }
       const bf16* sv = static_cast<const bf16*>(a.self_v) + (g.qs + r0 + row) * a.q_stride + h * DH;

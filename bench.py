@@ -72,11 +72,34 @@ def describe(w: W.Workload):
     }[w.name.replace("_subset", "")]
 
 
+# ----------------------------------------------------------------------------
+# Data-parallel pieces (weak scaling: every rank its own sequences, one
+# all-reduce of the flat fp32 gradient buffer per step, max-over-ranks time)
+# ----------------------------------------------------------------------------
+
+def rank_data_seed(rank: int) -> int:
+    """Seed of rank `rank`'s sequences; the weights come from the common seed."""
+    return 5 + 1000 * rank
+
+
+def allreduce_grads(flat, dist):
+    """Sums the ranks' gradient buffers in place (one collective per step)."""
+    dist.all_reduce(flat)
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time: the job's step time."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def make_workload(name, rank, batch=None):
     """The named workload; `batch` keeps only its first sequences (a small
     case of the same shapes, e.g. for profiler captures)."""
     if name == "training":
-        w = W.training(data_seed=5 + 1000 * rank)
+        w = W.training(data_seed=rank_data_seed(rank))
     else:
         w = W.WORKLOADS[name]()
     if batch is not None and batch < w.B:
@@ -261,7 +284,7 @@ def run_ours(args):
             ts.zero_grads()
             ts.run()
             if world > 1:
-                dist.all_reduce(ts.flat_grads)
+                allreduce_grads(ts.flat_grads, dist)
     else:
         def step():
             S.forward_stack(dw)
@@ -293,9 +316,7 @@ def run_ours(args):
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, dev)
 
     kern = {}
     for k, name in enumerate(H.KERNEL_NAMES):
@@ -392,7 +413,7 @@ def e2e_training(args, ts, dw, world, dist):
         ts.zero_grads()
         dx = ts.run()
         if world > 1:
-            dist.all_reduce(ts.flat_grads)
+            allreduce_grads(ts.flat_grads, dist)
         hdx.copy_(dx, non_blocking=True)
 
     step()
@@ -405,9 +426,7 @@ def e2e_training(args, ts, dw, world, dist):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
     if world > 1:
-        t = torch.tensor([ms], device=dw.x.device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, dw.x.device)
     return {"value": w.T * w.num_layers * world / (ms / 1000.0), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
 

@@ -159,6 +159,34 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+# kernel class -> the source file its traffic figure was captured from
+_KERNEL_SOURCES = {"attn_fwd": "attn_tc.cu", "attn_bwd": "attn_bwd_tc.cu"}
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` on the full training
+    workload, from the ncu capture summarised under profiles/ (a line
+    `traffic_per_full_launch_bytes: <kernel> <bytes> <source hash>`); None
+    when there is none or the kernel's source changed since the capture."""
+    import glob
+    import hashlib
+    src = _KERNEL_SOURCES.get(kernel)
+    if src is None or workload != "training":       # scaled to the full workload only
+        return None
+    path = os.path.join(ROOT, "hstu_sequential_transducer_b200", "csrc", src)
+    try:
+        digest = hashlib.sha256(open(path, "rb").read()).hexdigest()[:12]
+    except OSError:
+        return None
+    for md in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        for line in open(md):
+            parts = line.split()
+            if len(parts) == 4 and parts[0] == "traffic_per_full_launch_bytes:" and parts[1] == kernel:
+                if parts[3] == digest:
+                    return int(parts[2])
+    return None
+
+
 def read_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -339,8 +367,10 @@ def run_ours(args):
         "proj_out": ("tensor", 2 * w.T * d * d),
         "proj_in_bwd": ("tensor", 16 * w.T * d * d),
         "proj_out_bwd": ("tensor", 4 * w.T * d * d),
-        "ln_fwd": ("hbm", w.T * (6 * d + 8)),
-        "ln_bwd": ("hbm", w.T * (12 * d + 8)),
+        # read O (fp32) and U, write Z, row statistics
+        "ln_fwd": ("hbm", w.T * (8 * d + 8)),
+        # read dZ, O (fp32), U, Pre_U, statistics; write dO and dPre_U
+        "ln_bwd": ("hbm", w.T * (14 * d + 8)),
     }
     roof = None
     if kern:
@@ -358,7 +388,7 @@ def run_ours(args):
                 peak = peaks.get("hbm_gbs")
                 unit = "GB/s"
             roof = {"kernel": top, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
-                    "frac": ach / peak, "traffic": None,
+                    "frac": ach / peak, "traffic": profiled_traffic(top, w.name),
                     "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
                     "work_per_launch": work}
 

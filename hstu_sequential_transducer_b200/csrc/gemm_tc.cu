@@ -73,8 +73,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                    const __grid_constant__ CUtensorMap tmR, const KParams p) {
   using C = Cfg<BN, AK, BKM, EPI, TOUT>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Tiles need a 1024-byte aligned base; using the array itself (not an
+  // address rounded through an integer) keeps the pointers below in the
+  // shared state space, so staging accesses compile to shared, not generic,
+  // instructions.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {              // uniform over the block: all threads leave
+    if (threadIdx.x == 0 && p.status) atomicOr(p.status, kStatusSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* stages = smem;
   uint8_t* stg = smem + C::STAGES * C::STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(stg + C::NOUT * C::STG_BYTES);

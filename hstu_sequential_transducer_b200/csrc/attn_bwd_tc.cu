@@ -175,31 +175,71 @@ __device__ __forceinline__ int count_le_32(const long long* cts, long long tau) 
 // One 32-column chunk of the fast path: h = S/2 + bias/2 where columns
 // c >= p[k] add hd[k]; writes packed P and dS (unscaled) and accumulates the
 // total and the per-breakpoint suffix sums of dS.
+// Packed pairs of fp32 values (sm_100a f32x2 arithmetic).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 template <int NB, int E0 = 0, int NE = 32>
 __device__ __forceinline__ void bwd_chunk_fast(const uint32_t (&sr)[32], const uint32_t (&dr)[32],
                                                int c0, float hb, const int (&p)[2],
                                                const float (&hd)[2], uint32_t (&pk)[16],
                                                uint32_t (&dk)[16], float& tot, float (&suf)[2]) {
+  const uint64_t half2 = f2pack(0.5f, 0.5f), one2 = f2pack(1.f, 1.f), mone2 = f2pack(-1.f, -1.f);
+  const uint64_t hb2 = f2pack(hb, hb);
+  uint64_t tot2 = f2pack(0.f, 0.f), suf2[2] = {tot2, tot2};
 #pragma unroll
   for (int e = E0; e < E0 + NE; e += 2) {
-    float pa[2], ds[2];
+    const int c = c0 + e;
+    uint64_t h = f2fma(f2pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), half2, hb2);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int c = c0 + e + u;
-      float h = fmaf(__uint_as_float(sr[e + u]), 0.5f, hb);
+    for (int k = 0; k < NB; ++k)
+      h = f2add(h, f2pack(c >= p[k] ? hd[k] : 0.f, c + 1 >= p[k] ? hd[k] : 0.f));
+    float h0, h1;
+    f2unpack(h, h0, h1);
+    const uint64_t t = f2pack(tanh_fast(h0), tanh_fast(h1));
+    const uint64_t sg = f2fma(t, half2, half2);                  // sigmoid(x)
+    const uint64_t pa = f2fma(h, t, h);                          // SiLU(x)
+    const uint64_t w = f2mul(h, f2fma(t, mone2, one2));          // x (1 - sigmoid(x))
+    const uint64_t ds = f2mul(f2pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), f2fma(sg, w, sg));
+    tot2 = f2add(tot2, ds);
+    float d0, d1;
+    f2unpack(ds, d0, d1);
 #pragma unroll
-      for (int k = 0; k < NB; ++k) h += (c >= p[k]) ? hd[k] : 0.f;
-      const float t = tanh_fast(h);
-      const float sg = fmaf(t, 0.5f, 0.5f);
-      pa[u] = fmaf(h, t, h);                       // SiLU(x)
-      const float w = fmaf(-h, t, h);              // x (1 - sigmoid(x))
-      ds[u] = __uint_as_float(dr[e + u]) * fmaf(sg, w, sg);
-      tot += ds[u];
+    for (int k = 0; k < NB; ++k)
+      suf2[k] = f2add(suf2[k], f2pack(c >= p[k] ? d0 : 0.f, c + 1 >= p[k] ? d1 : 0.f));
+    float a0, a1;
+    f2unpack(pa, a0, a1);
+    pk[e / 2] = pack_bf16(a0, a1);
+    dk[e / 2] = pack_bf16(d0, d1);
+  }
+  float x0, x1;
+  f2unpack(tot2, x0, x1);
+  tot += x0 + x1;
 #pragma unroll
-      for (int k = 0; k < NB; ++k) suf[k] += (c >= p[k]) ? ds[u] : 0.f;
-    }
-    pk[e / 2] = pack_bf16(pa[0], pa[1]);
-    dk[e / 2] = pack_bf16(ds[0], ds[1]);
+  for (int k = 0; k < NB; ++k) {
+    f2unpack(suf2[k], x0, x1);
+    suf[k] += x0 + x1;
   }
 }
 

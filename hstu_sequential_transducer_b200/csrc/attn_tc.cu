@@ -201,6 +201,20 @@ __device__ __forceinline__ int time_bucket32(long long dt, int Bt) {
   return dt <= 0 ? 0 : min(64 - __clzll(dt), Bt - 1);
 }
 
+__device__ __forceinline__ int time_bucket_lo(uint32_t tq_lo, uint32_t tk_lo, int Bt) {
+  const int dt = (int)(tq_lo - tk_lo);
+  return dt <= 0 ? 0 : min(32 - __clz(dt), Bt - 1);
+}
+
+// Number of the 32 non-decreasing values cts[] that are <= tau.
+__device__ __forceinline__ int count_le32(const long long* cts, long long tau) {
+  int lo = 0;
+#pragma unroll
+  for (int step = 16; step >= 1; step >>= 1)
+    if (cts[lo + step - 1] <= tau) lo += step;
+  return lo + (cts[lo] <= tau ? 1 : 0);
+}
+
 // Number of the 128 non-decreasing values cts[] that are <= tau.
 __device__ __forceinline__ int count_le128(const long long* cts, long long tau) {
   if (cts[127] <= tau) return 128;
@@ -211,6 +225,26 @@ __device__ __forceinline__ int count_le128(const long long* cts, long long tau) 
   return lo;
 }
 
+// Packed pairs of fp32 values (sm_100a f32x2 arithmetic).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // Activation of one 32-column chunk in the fast path: h = S/2 + bias/2 with
 // the bias a step function (NB breakpoints, columns c < p[k] add hd[k]);
 // returns packed bf16 SiLU values.
@@ -218,18 +252,23 @@ template <int NB>
 __device__ __forceinline__ void act_chunk_fast(const uint32_t (&s)[32], int c0, float hb,
                                                const int (&p)[2], const float (&hd)[2],
                                                uint32_t (&pk)[16]) {
+  const uint64_t half2 = f2pack(0.5f, 0.5f), hb2 = f2pack(hb, hb);
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    float y[2];
+    const int c = c0 + e;
+    uint64_t h = f2fma(f2pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), half2, hb2);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int c = c0 + e + u;
-      float h = fmaf(__uint_as_float(s[e + u]), 0.5f, hb);
-#pragma unroll
-      for (int k = 0; k < NB; ++k) h += (c < p[k]) ? hd[k] : 0.f;
-      y[u] = silu_half(h);
-    }
-    pk[e / 2] = pack_bf16(y[0], y[1]);
+    for (int k = 0; k < NB; ++k)
+      h = f2add(h, f2pack(c < p[k] ? hd[k] : 0.f, c + 1 < p[k] ? hd[k] : 0.f));
+    float h0, h1;
+    f2unpack(h, h0, h1);
+    float t0, t1;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(h0));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(h1));
+    const uint64_t y = f2fma(h, f2pack(t0, t1), h);     // SiLU = h + h tanh(h)
+    float y0, y1;
+    f2unpack(y, y0, y1);
+    pk[e / 2] = pack_bf16(y0, y1);
   }
 }
 
@@ -565,25 +604,78 @@ __global__ void __launch_bounds__(352, 1)
           else if (nbw == 1) act_tile_fast<1>(sbuf, pbuf, hb, p, hd);
           else act_tile_fast<2>(sbuf, pbuf, hb, p, hd);
         } else {
+          const int last = max(min(kTile, kend - k0) - 1, 0);
+          const long long g_hi = tq - kts[0], g_lo = tq - kts[last];
+          const bool gap32 = __all_sync(0xffffffffu, !rvalid || (g_hi < 0x7fffffffLL && g_lo > -0x7fffffffLL));
+          const uint32_t tq_lo = (uint32_t)(unsigned long long)tq;
+          const uint32_t* kts_lo = reinterpret_cast<const uint32_t*>(kts);
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
+            const int c0 = c * 32;
             uint32_t sv[32], pk[16];
-            tmem_ld32(sbuf + c * 32, sv);
+            tmem_ld32(sbuf + c0, sv);
+            const int j0 = k0 + c0;
+            const bool masked = !rvalid || j0 >= kend || (!cand && j0 > qpos);
+            const bool visible = rvalid && j0 + 31 < kend && (cand || j0 + 31 <= qpos);
+            const bool cfar = qp_clamped - (j0 + 31) >= a.P - 1;
+            int cb_lo = 0, cnb = 3;
+            if (visible && cfar) {
+              cb_lo = time_bucket32(tq - kts[c0 + 31], a.Bt);
+              cnb = time_bucket32(tq - kts[c0], a.Bt) - cb_lo;
+            }
+            const bool all_masked = __all_sync(0xffffffffu, masked);
+            const bool cfast = __all_sync(0xffffffffu, visible && cfar && cnb <= 2);
             tmem_ld_wait();
+            if (all_masked) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float y[2];
+              for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            } else if (cfast) {
+              const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)cnb);
+              int p[2] = {0, 0};
+              float hd[2] = {0.f, 0.f};
 #pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int col = c * 32 + e + u;
-                const int jk = k0 + col;
-                const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
-                const int bp = min(max(qp_clamped - jk, 0), a.P - 1);
-                const int bt = time_bucket32(tq - kts[col], a.Bt);
-                const float h = 0.5f * (__uint_as_float(sv[e + u]) + rab[bp] + rab[32 + bt]);
-                y[u] = ok ? silu_half(h) : 0.f;
+              for (int k = 0; k < 2; ++k)
+                if (k < cnb) {
+                  const int b = cb_lo + 1 + k;
+                  p[k] = c0 + count_le32(kts + c0, tq - (1LL << (b - 1)));
+                  hd[k] = 0.5f * (rab[32 + b] - rab[32 + b - 1]);
+                }
+              const float hb = 0.5f * (rp_far + rab[32 + cb_lo]);
+              if (nbw == 0) act_chunk_fast<0>(sv, c0, hb, p, hd, pk);
+              else if (nbw == 1) act_chunk_fast<1>(sv, c0, hb, p, hd, pk);
+              else act_chunk_fast<2>(sv, c0, hb, p, hd, pk);
+            } else if (gap32) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float y[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                  const int col = c * 32 + e + u;
+                  const int jk = k0 + col;
+                  const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
+                  const int bp = min(max(qp_clamped - jk, 0), a.P - 1);
+                  const int bt = time_bucket_lo(tq_lo, kts_lo[2 * col], a.Bt);
+                  const float h = 0.5f * (__uint_as_float(sv[e + u]) + rab[bp] + rab[32 + bt]);
+                  y[u] = ok ? silu_half(h) : 0.f;
+                }
+                pk[e / 2] = pack_bf16(y[0], y[1]);
               }
-              pk[e / 2] = pack_bf16(y[0], y[1]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float y[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                  const int col = c * 32 + e + u;
+                  const int jk = k0 + col;
+                  const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
+                  const int bp = min(max(qp_clamped - jk, 0), a.P - 1);
+                  const int bt = time_bucket32(tq - kts[col], a.Bt);
+                  const float h = 0.5f * (__uint_as_float(sv[e + u]) + rab[bp] + rab[32 + bt]);
+                  y[u] = ok ? silu_half(h) : 0.f;
+                }
+                pk[e / 2] = pack_bf16(y[0], y[1]);
+              }
             }
             tmem_st16(pbuf + c * 16, pk);
           }

@@ -697,13 +697,15 @@ int sms();
 // (each warpgroup transposes its 32 queries into a dense fp32 tile in shared
 // memory and adds it to the fp32 dQ accumulator with one TMA bulk reduce-add;
 // rows past the sequence end carry exact zeros).  Q/dO blocks come through a
-// two-stage ring that the producer keeps prefetched into L2.  The layout packs
+// three-stage ring that the producer keeps prefetched into L2, so block g+1's
+// loads overlap block g-1's dV/dK; the P^T and dS tiles are single-buffered
+// (block g is written once block g-1's MMAs have read them).  The layout packs
 // almost the whole 227 KB budget, so the kernel relies on a 1024-byte aligned
 // dynamic shared memory base (checked; it reports kStatusSmemAlign if not).
 // TMEM: S^T [0,64) dP^T [64,128) dQ^T_0 [128,192) dQ^T_1 [192,256)
 //       dV [256,384) dK [384,512)
 constexpr int kQB = 64;
-constexpr int kQStages = 2;
+constexpr int kQStages = 3;
 
 struct B3Cfg {
   static constexpr int DH = 128;
@@ -714,7 +716,7 @@ struct B3Cfg {
   static constexpr int PS_BYTES = kT * kQB * 2;        // P^T or dS [key][query] for one block = 16 KB
   static constexpr int DQ_BYTES = kQB * DH * 4;        // dQ staging, 2 x [32 queries][dh] fp32 = 32 KB
   static constexpr int BAR_BYTES = 1536;               // barriers, rab tables, TMEM slot
-  static constexpr int SMEM = 2 * KTILE + kQStages * QSTAGE + 4 * PS_BYTES + DQ_BYTES + kQStages * TS_BYTES +
+  static constexpr int SMEM = 2 * KTILE + kQStages * QSTAGE + 2 * PS_BYTES + DQ_BYTES + kQStages * TS_BYTES +
                               BAR_BYTES;
   static constexpr uint32_t IDESC_ST = idesc_bf16(128, kQB, false, false);   // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DKV = idesc_bf16(128, DH, false, true);    // P^T dO, dS^T Q
@@ -740,25 +742,25 @@ __global__ void __launch_bounds__(kBThreads, 1)
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::KTILE;
   uint8_t* sQD = sV + C::KTILE;                    // kQStages x (Q | dO)
-  uint8_t* sPT = sQD + kQStages * C::QSTAGE;        // 2 x P^T
-  uint8_t* sDS = sPT + 2 * C::PS_BYTES;             // 2 x dS
-  float* sDQ = reinterpret_cast<float*>(sDS + 2 * C::PS_BYTES);   // 2 x dQ staging [32][128]
-  uint8_t* sTS = sDS + 2 * C::PS_BYTES + C::DQ_BYTES;             // kQStages x times
+  uint8_t* sPT = sQD + kQStages * C::QSTAGE;        // P^T
+  uint8_t* sDS = sPT + C::PS_BYTES;                 // dS
+  float* sDQ = reinterpret_cast<float*>(sDS + C::PS_BYTES);   // 2 x dQ staging [32][128]
+  uint8_t* sTS = sDS + C::PS_BYTES + C::DQ_BYTES;             // kQStages x times
   uint64_t* bars = reinterpret_cast<uint64_t*>(sTS + kQStages * C::TS_BYTES);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* qd_full = bars + 2;                     // [2]
-  uint64_t* qd_empty = bars + 4;                    // [2]
+  uint64_t* qd_full = bars + 2;                     // [3] (slots 2..4)
+  uint64_t* qd_empty = bars + 19;                   // [3] (slots 19..21)
   uint64_t* st_full = bars + 6;                     // S^T, dP^T of the current block are in TMEM
   uint64_t* s_free = bars + 7;                      // (8 warps) ... and have been read
-  uint64_t* pds_full = bars + 8;                    // [2] (8 warps) P^T, dS of a block are in smem
-  uint64_t* ps_free = bars + 10;                    // [2] the block's MMAs have read them
+  uint64_t* pds_full = bars + 8;                    // (8 warps) P^T, dS of the block are in smem
+  uint64_t* ps_free = bars + 10;                    // the block's MMAs have read them
   uint64_t* dq_full = bars + 12;                    // [2] dQ^T of a block is in TMEM
   uint64_t* dq_free = bars + 14;                    // [2] (8 warps) ... and has been read
   uint64_t* dkv_full = bars + 16;
   uint64_t* dkv_free = bars + 17;                   // (8 warps)
   uint64_t* done_bar = bars + 18;
-  float* rab = reinterpret_cast<float*>(bars + 20);  // [2][64] per warpgroup
+  float* rab = reinterpret_cast<float*>(bars + 24);  // [2][64] per warpgroup
   float* drab = rab + 128;                           // [2][64] per warpgroup
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drab + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -768,7 +770,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const int total = *P.w.total;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 19; ++i) {
+    for (int i = 0; i < 22; ++i) {
       const bool act = (i == 7 || i == 8 || i == 9 || i == 14 || i == 15 || i == 17);
       mbar_init(&bars[i], act ? kActWarps : 1);
     }
@@ -911,11 +913,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
             const uint32_t gp = g + m - 1, b = gp & 1;
             const int st = (int)(gp % kQStages);
             if (m == 1 && !mbar_wait(dkv_free, (items_done & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
-            if (!mbar_wait(&pds_full[b], (gp >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            if (!mbar_wait(pds_full, gp & 1, abort_flag, P.status)) { ok = false; break; }
             if (gp >= 2 && !mbar_wait(&dq_free[b], ((gp - 2) >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t q_s = smem_u32(sQD + st * C::QSTAGE), do_s = q_s + C::QTILE;
-            const uint32_t pt_s = smem_u32(sPT + b * C::PS_BYTES), ds_s = smem_u32(sDS + b * C::PS_BYTES);
+            const uint32_t pt_s = smem_u32(sPT), ds_s = smem_u32(sDS);
             const uint32_t acc0 = m > 1 ? 1u : 0u;
 #pragma unroll
             for (int k = 0; k < kQB / 16; ++k)
@@ -931,7 +933,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
               mma_ss(tQ(b), sdesc_mnmajor(k_s + k * 2048, kT * 128), sdesc_mnmajor(ds_s + k * 2048, kT * 128),
                      C::IDESC_DQT, k > 0 ? 1u : 0u);
             mma_commit(&dq_full[b]);
-            mma_commit(&ps_free[b]);
+            mma_commit(ps_free);
           }
         }
         if (!ok) break;
@@ -1143,9 +1145,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
           add_t(b_lo + nb, below);
         }
         // P^T and dS into this block's tiles once block gb-2's MMAs have read them
-        if (gb >= 2) fail = !mbar_wait(&ps_free[b], ((gb - 2) >> 1) & 1, abort_flag, P.status) || fail;
-        uint8_t* ptb = sPT + b * C::PS_BYTES;
-        uint8_t* dsb = sDS + b * C::PS_BYTES;
+        if (gb >= 1) fail = !mbar_wait(ps_free, (gb - 1) & 1, abort_flag, P.status) || fail;
+        uint8_t* ptb = sPT;
+        uint8_t* dsb = sDS;
 #pragma unroll
         for (int g8 = 0; g8 < 4; ++g8) {
           const uint32_t off = mn_off(row, wg * 32 + g8 * 8, kT * 128);
@@ -1154,7 +1156,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&pds_full[b]);
+        if (lane == 0) mbar_arrive(pds_full);
         // the previous block's dQ^T (its MMAs ran while this block was computed)
         if (m >= 1) drain(gb - 1, q0 - kQB);
       }

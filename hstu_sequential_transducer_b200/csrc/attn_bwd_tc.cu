@@ -1144,7 +1144,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
             }
           add_t(b_lo + nb, below);
         }
-        // P^T and dS into this block's tiles once block gb-2's MMAs have read them
+        // P^T and dS into the tiles once block gb-1's MMAs have read them
         if (gb >= 1) fail = !mbar_wait(ps_free, (gb - 1) & 1, abort_flag, P.status) || fail;
         uint8_t* ptb = sPT;
         uint8_t* dsb = sDS;

@@ -12,9 +12,12 @@
 //   warp 0      TMA producer: 128x64 A and BNx64 B tiles into a ring of stages
 //   warp 1      MMA issuer: 4 x tcgen05.mma (128 x BN x 16) per stage into a
 //               double-buffered TMEM accumulator
-//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, bias / SiLU /
-//               residual, 128-byte-swizzled staging in shared memory, TMA store
-//               (or TMA reduce-add for split-K)
+//   warps 2..9  epilogue, two warpgroups taking alternate 128-byte-wide
+//               chunks of each tile: tcgen05.ld of their 32 TMEM lanes, bias /
+//               SiLU / residual, 128-byte-swizzled staging in shared memory
+//               (one staging tile per warpgroup), TMA store (or TMA reduce-add
+//               for split-K); a warpgroup waits for its previous store only
+//               when it next needs its staging tile
 // Every mbarrier wait is bounded; a timeout sets the library's device status
 // word and the CTA drains its own copies and MMAs, frees its TMEM and exits.
 #include <cuda.h>
@@ -30,7 +33,7 @@ using namespace tc;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kMaxSmem = 232448;
 
 template <int BN, bool AK, bool BKM, int EPI, typename TOUT>
@@ -43,9 +46,9 @@ struct Cfg {
   static constexpr int CW = 128 / OUT_ES;  // columns per staged chunk (128 bytes per row)
   static constexpr int STG_BYTES = BM * 128;
   static constexpr int BAR_BYTES = 1024;
-  static constexpr int STAGES_FIT = (kMaxSmem - 1024 - NOUT * STG_BYTES - BAR_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = (kMaxSmem - 1024 - 2 * NOUT * STG_BYTES - BAR_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static constexpr int SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + NOUT * STG_BYTES + BAR_BYTES;
+  static constexpr int SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 2 * NOUT * STG_BYTES + BAR_BYTES;
   static constexpr uint32_t IDESC = idesc_bf16(BM, BN, !AK, !BKM);
   static_assert(STAGES >= 2, "not enough shared memory for two stages");
   static_assert(BN % CW == 0 || CW > BN, "chunking");
@@ -62,6 +65,14 @@ struct KParams {
   uint32_t* status;
   bool has_c;           // SILU_SPLIT: write Pre too
 };
+
+// SiLU(x) = h + h tanh(h) with h = x / 2 (x sigmoid(x), as an identity).
+__device__ __forceinline__ float silu_tanh(float x) {
+  const float h = 0.5f * x;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
 
 __device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
@@ -85,13 +96,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw;
   uint8_t* stages = smem;
   uint8_t* stg = smem + C::STAGES * C::STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + C::NOUT * C::STG_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + 2 * C::NOUT * C::STG_BYTES);
   uint64_t* full = bars;                       // [STAGES]
   uint64_t* empty = bars + C::STAGES;          // [STAGES]
   uint64_t* acc_full = empty + C::STAGES;      // [2]
   uint64_t* acc_empty = acc_full + 2;          // [2]
-  uint64_t* res_bar = acc_empty + 2;           // [1]
-  uint64_t* done_bar = res_bar + 1;            // [1]
+  uint64_t* res_bar = acc_empty + 2;           // [2] one per epilogue warpgroup
+  uint64_t* done_bar = res_bar + 2;            // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -105,9 +116,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], 8);
     }
-    mbar_init(res_bar, 1);
+    mbar_init(&res_bar[0], 1);
+    mbar_init(&res_bar[1], 1);
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -217,8 +229,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;             // chunks half, half + 2, ...
     const int row = quarter * 32 + lane;          // accumulator row (TMEM lane)
-    const int et = threadIdx.x - 64;              // 0..127
+    const int et = (threadIdx.x - 64) & 127;      // thread in the warpgroup
+    const uint32_t bid = 1 + half;                // this warpgroup's named barrier
+    uint8_t* const wstg = stg + half * C::NOUT * C::STG_BYTES;
+    uint64_t* const wres = res_bar + half;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -228,19 +244,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m0 = (tile / p.n_tiles) * BM, n0 = (tile % p.n_tiles) * BN;
       bool fail = *abort_flag != 0;
       if (!fail) fail = !mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status);
-      if (named_barrier_any(1, 128, fail)) break;
+      if (named_barrier_any(bid, 128, fail)) break;
       tc_fence_after();
       const uint32_t t_acc = tmem_base + lane_off + acc * BN;
       bool ok = true;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += C::CW) {
+      for (int c0 = half * C::CW; c0 < BN; c0 += 2 * C::CW) {
         if (c0 >= p.N - n0) break;   // chunk entirely past N
-        if (EPI == EPI_RESID) {
-          if (et == 0) {
-            mbar_expect_tx(res_bar, C::STG_BYTES);
-            tma_load_2d(stg, &tmR, res_bar, n0 + c0, m0);
-          }
-        }
         float v[C::CW];
         {
           uint32_t r[32];
@@ -260,10 +270,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             v[i] += n < p.N ? bf16_bits_to_f(__ldg(b16 + n)) : 0.f;
           }
         }
+        // the staging tile is free once this warpgroup's previous store has read it
+        if (et == 0) bulk_wait_read0();
+        named_barrier(bid, 128);
         if (EPI == EPI_RESID) {
-          const bool fail_r = !mbar_wait(res_bar, res_phase, abort_flag, p.status);
+          if (et == 0) {
+            mbar_expect_tx(wres, C::STG_BYTES);
+            tma_load_2d(wstg, &tmR, wres, n0 + c0, m0);
+          }
+          const bool fail_r = !mbar_wait(wres, res_phase, abort_flag, p.status);
           res_phase ^= 1;
-          if (named_barrier_any(1, 128, fail_r)) {
+          if (named_barrier_any(bid, 128, fail_r)) {
             ok = false;
             break;
           }
@@ -279,11 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 4; ++q) {
               const float x0 = v[8 * j + 2 * q], x1 = v[8 * j + 2 * q + 1];
               pp[q] = pack_bf16(x0, x1);
-              const float s0 = x0 / (1.f + __expf(-x0)), s1 = x1 / (1.f + __expf(-x1));
-              gg[q] = pack_bf16(s0, s1);
+              gg[q] = pack_bf16(silu_tanh(x0), silu_tanh(x1));
             }
-            *reinterpret_cast<uint4*>(stg + sw128(row, j)) = g;
-            *reinterpret_cast<uint4*>(stg + C::STG_BYTES + sw128(row, j)) = pre;
+            *reinterpret_cast<uint4*>(wstg + sw128(row, j)) = g;
+            *reinterpret_cast<uint4*>(wstg + C::STG_BYTES + sw128(row, j)) = pre;
           }
         } else if (C::OUT_ES == 2) {
 #pragma unroll
@@ -291,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint4 o;
             uint32_t* oo = reinterpret_cast<uint32_t*>(&o);
             if (EPI == EPI_RESID) {
-              const uint4 rr = *reinterpret_cast<const uint4*>(stg + sw128(row, j));
+              const uint4 rr = *reinterpret_cast<const uint4*>(wstg + sw128(row, j));
               const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rr);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
@@ -302,34 +318,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int q = 0; q < 4; ++q) oo[q] = pack_bf16(v[8 * j + 2 * q], v[8 * j + 2 * q + 1]);
             }
-            *reinterpret_cast<uint4*>(stg + sw128(row, j)) = o;
+            *reinterpret_cast<uint4*>(wstg + sw128(row, j)) = o;
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             if (EPI == EPI_RESID) {
-              const float4 rr = *reinterpret_cast<const float4*>(stg + sw128(row, j));
+              const float4 rr = *reinterpret_cast<const float4*>(wstg + sw128(row, j));
               o.x += rr.x; o.y += rr.y; o.z += rr.z; o.w += rr.w;
             }
-            *reinterpret_cast<float4*>(stg + sw128(row, j)) = o;
+            *reinterpret_cast<float4*>(wstg + sw128(row, j)) = o;
           }
         }
         fence_proxy_async_smem();
-        named_barrier(1, 128);
+        named_barrier(bid, 128);
         if (et == 0) {
           if (EPI == EPI_ATOMIC_F32) {
-            tma_reduce_add_2d(&tmC, stg, n0 + c0, m0);
+            tma_reduce_add_2d(&tmC, wstg, n0 + c0, m0);
           } else if (EPI == EPI_SILU_SPLIT) {
-            tma_store_2d(&tmC2, stg, n0 + c0, m0);
-            if (p.has_c) tma_store_2d(&tmC, stg + C::STG_BYTES, n0 + c0, m0);
+            tma_store_2d(&tmC2, wstg, n0 + c0, m0);
+            if (p.has_c) tma_store_2d(&tmC, wstg + C::STG_BYTES, n0 + c0, m0);
           } else {
-            tma_store_2d(&tmC, stg, n0 + c0, m0);
+            tma_store_2d(&tmC, wstg, n0 + c0, m0);
           }
           bulk_commit();
-          bulk_wait_read0();
         }
-        named_barrier(1, 128);
       }
       if (!ok) break;
       // accumulator buffer free for the MMA warp

@@ -146,6 +146,13 @@ __device__ __forceinline__ float tanh_fast(float x) {
 }
 
 constexpr int kBThreads = 320;
+
+// SiLU'(x) = sigma(x) (1 + x (1 - sigma(x))) with sigma(x) = (1 + tanh(x/2)) / 2
+__device__ __forceinline__ float silu_grad_fast(float x) {
+  const float h = 0.5f * x;
+  const float t = tanh_fast(h);
+  return 0.5f * (1.f + t + fmaf(-h * t, t, h));
+}
 constexpr int kPrefetch = 4;   // query blocks the backward producer prefetches ahead
 constexpr int kActWarps = 8;
 
@@ -693,10 +700,15 @@ int sms();
 // dK += dS^T Q and as the MN-major B operand of dQ^T_g = K^T dS^T.  dQ^T has a
 // double buffer of its own in TMEM, so the next block's S^T, dP^T never wait
 // for the dQ drain: S^T(g+1) is issued as soon as block g's scores are in
-// registers, and the activation warps drain dQ^T(g-1) after finishing block g
-// (each warpgroup transposes its 32 queries into a dense fp32 tile in shared
-// memory and adds it to the fp32 dQ accumulator with one TMA bulk reduce-add;
-// rows past the sequence end carry exact zeros).  Q/dO blocks come through a
+// registers.  A warpgroup of its own drains dQ^T(g) (transposes it into a
+// dense fp32 tile in shared memory and adds it to the fp32 dQ accumulator
+// with TMA bulk reduce-adds; rows past the sequence end carry exact zeros),
+// so the activation warps go from one block to the next without it; they
+// also finish an item with dK, dV times SiLU'(Pre) into dPre, with the Pre
+// loads in flight during the TMEM loads, while the producer has the next
+// item's K and V tiles prefetched into L2.  Off the fast path, a warp whose 32
+// columns hold no allowed pair writes zeros, and time gaps within +-2^31 s
+// take 32-bit bucket arithmetic.  Q/dO blocks come through a
 // three-stage ring that the producer keeps prefetched into L2, so block g+1's
 // loads overlap block g-1's dV/dK; the P^T and dS tiles are single-buffered
 // (block g is written once block g-1's MMAs have read them).  The layout packs
@@ -726,7 +738,19 @@ struct B3Cfg {
 // query blocks that see key tile kt: from its first key to the end
 __device__ __forceinline__ int qblocks(int n, int kt) { return (n - kt * kT + kQB - 1) / kQB; }
 
-__global__ void __launch_bounds__(kBThreads, 1)
+// Warp roles of the dh = 128 kernel: warpgroup 0 = producer (warp 0), MMA
+// issuer (warp 1), two idle warps; warpgroups 1 and 2 = key-row warps;
+// warpgroup 3 = dQ drain.  The 65,536 registers of the launch (512 threads x
+// 128) are re-split with setmaxnreg: 9,216 + 2 x 22,528 + 10,240.
+constexpr int kB3Threads = 512;
+constexpr int kRegCtl = 72, kRegAct = 176, kRegDrain = 80;
+static_assert(128 * (kRegCtl + 2 * kRegAct + kRegDrain) <= 65536, "register split");
+template <int R>
+__device__ __forceinline__ void reg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R)); }
+template <int R>
+__device__ __forceinline__ void reg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R)); }
+
+__global__ void __launch_bounds__(kB3Threads, 1)
     attn_bwd_tc3_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                         const __grid_constant__ CUtensorMap tmdQ, const BParams P) {
@@ -771,8 +795,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 22; ++i) {
-      const bool act = (i == 7 || i == 8 || i == 9 || i == 14 || i == 15 || i == 17);
-      mbar_init(&bars[i], act ? kActWarps : 1);
+      const bool act = (i == 7 || i == 8 || i == 9 || i == 17);
+      const bool drn = (i == 14 || i == 15);
+      mbar_init(&bars[i], act ? kActWarps : drn ? 4 : 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -786,6 +811,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
   auto tQ = [tmem](uint32_t b) { return tmem + 128u + b * 64u; };
   const uint32_t tdV = tmem + 256, tdK = tmem + 384;
 
+  if (warp < 4) {
+  reg_dec<kRegCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     uint32_t items_done = 0, g = 0;
@@ -812,6 +839,17 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         kv_iss = true;
         kv_par = items_done & 1;
+        // the next item's K and V wait for this item's last MMA: have them in L2
+        const int itn = it + gridDim.x;
+        if (itn < total) {
+          const BItem nx = P.w.items[itn];
+          const int32_t kr = (int32_t)(a.q_offsets[nx.b] + nx.kt * kT);
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            tma_prefetch_2d(&tmK, nx.h * DH + 64 * x, kr);
+            tma_prefetch_2d(&tmV, nx.h * DH + 64 * x, kr);
+          }
+        }
       }
       ++items_done;
       // L2 prefetch keeps the Q, dO and time rows kPrefetch blocks ahead of
@@ -946,10 +984,60 @@ __global__ void __launch_bounds__(kBThreads, 1)
       volatile int never = 0;
       mbar_wait(done_bar, 0, &never, P.status);
     }
+  }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ dQ drain
+    reg_dec<kRegDrain>();
+    // per block: dQ^T (dh rows on TMEM lanes, 64 query columns) times 1/N,
+    // transposed into the staging tile, one bulk reduce-add per 32 queries
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;             // dh row (dQ^T lane)
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int tw = threadIdx.x & 127;
+    const float inv_N = a.inv_N;
+    uint32_t g = 0;
+    bool fail = false;
+    for (int it = blockIdx.x; it < total && !fail; it += gridDim.x) {
+      const BItem item = P.w.items[it];
+      int64_t s0;
+      int n, hlen;
+      bgeom(a, item.b, s0, n, hlen);
+      const int k0 = item.kt * kT;
+      const int nqb = qblocks(n, item.kt);
+      for (int m = 0; m < nqb; ++m) {
+        const uint32_t gb = g + m, b = gb & 1;
+        const bool f = !mbar_wait(&dq_full[b], (gb >> 1) & 1, abort_flag, P.status);
+        if (tw == 0) bulk_wait_read0();             // the previous block's reduces have read the staging tile
+        if (named_barrier_any(4, 128, f)) { fail = true; break; }
+        tc_fence_after();
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tQ(b) + lane_off, r0);
+        tmem_ld32(tQ(b) + lane_off + 32, r1);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dq_free[b]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sDQ[i * DH + row] = __uint_as_float(r0[i]) * inv_N;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sDQ[(32 + i) * DH + row] = __uint_as_float(r1[i]) * inv_N;
+        fence_proxy_async_smem();
+        named_barrier(4, 128);
+        if (tw == 0) {
+          const int32_t q = (int32_t)(s0 + k0 + m * kQB);
+          tma_reduce_add_2d(&tmdQ, sDQ, item.h * DH, q);
+          tma_reduce_add_2d(&tmdQ, sDQ + 32 * DH, item.h * DH, q + 32);
+          bulk_commit();
+        }
+      }
+      g += nqb;
+    }
+    if (tw == 0) bulk_wait0();
   } else {
     // ------------------------------------------------------------ key-row warps
+    reg_inc<kRegAct>();
     const int quarter = warp & 3;
-    const int wg = (warp - 2) >> 2;                  // query columns [32 wg, 32 wg + 32) of a block
+    const int wg = (warp - 4) >> 2;                  // query columns [32 wg, 32 wg + 32) of a block
     const int row = quarter * 32 + lane;             // key in the tile (S^T lane) / dh row (dQ^T lane)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     // The two warpgroups run independently: each has its own rab table, bucket
@@ -961,7 +1049,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     uint32_t items_done = 0, g = 0;
     int cur_h = -1;
     const float inv_N = a.inv_N;
-    const int tw = (threadIdx.x - 64) & 127;          // thread in the warpgroup
+    const int tw = threadIdx.x & 127;                 // thread in the warpgroup
     bool fail = false;
     for (int it = blockIdx.x; it < total && !fail; it += gridDim.x) {
       const BItem item = P.w.items[it];
@@ -1023,42 +1111,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         p_sum += v;
       };
-      // drain this warpgroup's 32 queries of dQ^T of block gd (query rows
-      // q0d ..): read its TMEM buffer and release it, transpose into the
-      // warpgroup's staging half, one bulk reduce-add into dQ.  A failed wait
-      // only marks `fail`; the warpgroup stops together at its next barrier.
-      float* sdq = sDQ + wg * (32 * DH);
-      auto drain = [&](uint32_t gd, int q0d) {
-        const uint32_t b = gd & 1;
-        bool f = !mbar_wait(&dq_full[b], (gd >> 1) & 1, abort_flag, P.status);
-        if (tw == 0) bulk_wait_read0();             // the previous reduce has read the staging half
-        if (named_barrier_any(bid, 128, f)) {
-          fail = true;
-          return;
-        }
-        tc_fence_after();
-        uint32_t r[32];
-        tmem_ld32(tQ(b) + lane_off + wg * 32, r);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dq_free[b]);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sdq[i * DH + row] = __uint_as_float(r[i]) * inv_N;
-        fence_proxy_async_smem();
-        named_barrier(bid, 128);
-        if (tw == 0) {
-          tma_reduce_add_2d(&tmdQ, sdq, item.h * DH, (int32_t)(s0 + q0d + wg * 32));
-          bulk_commit();
-        }
-      };
-
       for (int m = 0; m < nqb; ++m) {
         const uint32_t gb = g + m, b = gb & 1;
         const int st = (int)(gb % kQStages);
         const int q0 = k0 + m * kQB;
         fail = !mbar_wait(st_full, gb & 1, abort_flag, P.status) || fail;
-        if (named_barrier_any(bid, 128, fail)) { fail = true; break; }
         tc_fence_after();
         // S^T, dP^T loads in flight while the path is chosen
         uint32_t sr[32], dr[32], pk[16], dk[16];
@@ -1074,6 +1131,18 @@ __global__ void __launch_bounds__(kBThreads, 1)
           nb = tb64(qts[wg * 32 + 31] - tk, a.Bt) - b_lo;
         }
         const bool fast = __all_sync(0xffffffffu, full && far && nb <= 2);
+        // off the fast path: a warp with no allowed pair in its 32 columns
+        // writes zeros; gaps within +-2^31 s take 32-bit bucket arithmetic
+        const int lastc = min(31, n - 1 - qf);
+        const bool any_t = kvalid && lastc >= 0 && (qf + lastc >= hlen || jk <= qf + lastc);
+        bool g32_t = true;
+        if (!fast && any_t) {
+          const long long dlo = qts[wg * 32] - tk, dhi = qts[wg * 32 + lastc] - tk;
+          g32_t = dlo > -(1LL << 31) && dhi < (1LL << 31);
+        }
+        const bool anyok = __any_sync(0xffffffffu, any_t);
+        const bool g32 = __all_sync(0xffffffffu, g32_t);
+        const uint32_t tk32 = (uint32_t)tk;
         tmem_ld_wait();
         // the scores are in registers: the next block's may overwrite them
         tc_fence_before();
@@ -1102,6 +1171,41 @@ __global__ void __launch_bounds__(kBThreads, 1)
             if (nbw == 0) bwd_chunk_fast<0, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
             else if (nbw == 1) bwd_chunk_fast<1, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
             else bwd_chunk_fast<2, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
+            return;
+          }
+          if (!anyok) {
+#pragma unroll
+            for (int e = E0; e < E0 + 16; e += 2) pk[e / 2] = dk[e / 2] = 0u;
+            return;
+          }
+          if (g32) {
+#pragma unroll
+            for (int e = E0; e < E0 + 16; e += 2) {
+              float pv[2], dv[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int col = wg * 32 + e + u;
+                const int qpos = q0 + col;
+                const bool ok = kvalid && qpos < n && (qpos >= hlen || jk <= qpos);
+                const int bp = min(max(min(qpos, hlen) - jk, 0), a.P - 1);
+                const int dt = (int)((uint32_t)qts[col] - tk32);
+                const int bt = dt <= 0 ? 0 : min(32 - __clz(dt), a.Bt - 1);
+                const float h = 0.5f * (__uint_as_float(sr[e + u]) + rabw[bp] + rabw[32 + bt]);
+                const float t = tanh_fast(h);
+                const float sg = fmaf(t, 0.5f, 0.5f);
+                const float pa = ok ? fmaf(h, t, h) : 0.f;
+                const float ds = ok ? __uint_as_float(dr[e + u]) * fmaf(sg, fmaf(-h, t, h), sg) : 0.f;
+                if (ok) {
+                  if (bp < a.P - 1) atomicAdd(&drabw[bp], ds);
+                  else far_sum += ds;
+                  add_t(bt, ds);
+                }
+                pv[u] = pa;
+                dv[u] = ds;
+              }
+              pk[e / 2] = pack_bf16(pv[0], pv[1]);
+              dk[e / 2] = pack_bf16(dv[0], dv[1]);
+            }
             return;
           }
 #pragma unroll
@@ -1157,11 +1261,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(pds_full);
-        // the previous block's dQ^T (its MMAs ran while this block was computed)
-        if (m >= 1) drain(gb - 1, q0 - kQB);
       }
-      if (fail) break;
-      if (nqb >= 1) drain(g + nqb - 1, k0 + (nqb - 1) * kQB);
+      // a failed wait (the kernel is aborting) ends the item loop for the
+      // whole warpgroup together
+      if (named_barrier_any(bid, 128, fail)) { fail = true; break; }
       // flush this key row's bucket sums
       if (tb_cur >= 0) atomicAdd(&drabw[32 + tb_cur], t_sum);
       if (pb_cur >= 0) atomicAdd(&drabw[pb_cur], p_sum);
@@ -1183,15 +1286,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
         uint32_t rv[32], rk[32];
         tmem_ld32(tdV + lane_off + c * 32, rv);
         tmem_ld32(tdK + lane_off + c * 32, rk);
+        const int col = item.h * DH + c * 32;
+        uint4 pv4[4], pk4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          pv4[i] = kvalid ? *reinterpret_cast<const uint4*>(pre + rowoff + d + col + 8 * i) : make_uint4(0, 0, 0, 0);
+          pk4[i] = kvalid ? *reinterpret_cast<const uint4*>(pre + rowoff + 3 * d + col + 8 * i) : make_uint4(0, 0, 0, 0);
+        }
         tmem_ld_wait();
         if (kvalid) {
-          const int col = item.h * DH + c * 32;
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            const uint4 pv4 = *reinterpret_cast<const uint4*>(pre + rowoff + d + col + i);
-            const uint4 pk4 = *reinterpret_cast<const uint4*>(pre + rowoff + 3 * d + col + i);
-            const __nv_bfloat162* pvh = reinterpret_cast<const __nv_bfloat162*>(&pv4);
-            const __nv_bfloat162* pkh = reinterpret_cast<const __nv_bfloat162*>(&pk4);
+          for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162* pvh = reinterpret_cast<const __nv_bfloat162*>(&pv4[i]);
+            const __nv_bfloat162* pkh = reinterpret_cast<const __nv_bfloat162*>(&pk4[i]);
             uint4 ov, ok4;
             uint32_t* ovw = reinterpret_cast<uint32_t*>(&ov);
             uint32_t* okw = reinterpret_cast<uint32_t*>(&ok4);
@@ -1199,13 +1306,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
             for (int u = 0; u < 4; ++u) {
               const float2 fv = __bfloat1622float2(pvh[u]);
               const float2 fk = __bfloat1622float2(pkh[u]);
-              ovw[u] = pack_bf16(__uint_as_float(rv[i + 2 * u]) * inv_N * silu_grad_acc(fv.x),
-                                 __uint_as_float(rv[i + 2 * u + 1]) * inv_N * silu_grad_acc(fv.y));
-              okw[u] = pack_bf16(__uint_as_float(rk[i + 2 * u]) * inv_N * silu_grad_acc(fk.x),
-                                 __uint_as_float(rk[i + 2 * u + 1]) * inv_N * silu_grad_acc(fk.y));
+              const int j = 8 * i + 2 * u;
+              ovw[u] = pack_bf16(__uint_as_float(rv[j]) * inv_N * silu_grad_fast(fv.x),
+                                 __uint_as_float(rv[j + 1]) * inv_N * silu_grad_fast(fv.y));
+              okw[u] = pack_bf16(__uint_as_float(rk[j]) * inv_N * silu_grad_fast(fk.x),
+                                 __uint_as_float(rk[j + 1]) * inv_N * silu_grad_fast(fk.y));
             }
-            *reinterpret_cast<uint4*>(dpre + rowoff + d + col + i) = ov;
-            *reinterpret_cast<uint4*>(dpre + rowoff + 3 * d + col + i) = ok4;
+            *reinterpret_cast<uint4*>(dpre + rowoff + d + col + 8 * i) = ov;
+            *reinterpret_cast<uint4*>(dpre + rowoff + 3 * d + col + 8 * i) = ok4;
           }
         }
       }
@@ -1221,7 +1329,6 @@ __global__ void __launch_bounds__(kBThreads, 1)
       const int bi = tw & 31;
       if (dst && bi < nb && drabw[tw] != 0.f) atomicAdd(dst + cur_h * nb + bi, drabw[tw] * inv_N);
     }
-    if (tw == 0) bulk_wait0();
   }
 
   tc_fence_before();
@@ -1303,7 +1410,7 @@ cudaError_t launch_bwd3(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaSt
   P.status = status;
   e = cudaFuncSetAttribute(attn_bwd_tc3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  attn_bwd_tc3_kernel<<<sms(), kBThreads, C::SMEM, s>>>(tQ, tK, tV, tdO, tdQ, P);
+  attn_bwd_tc3_kernel<<<sms(), kB3Threads, C::SMEM, s>>>(tQ, tK, tV, tdO, tdQ, P);
   count_launch();
   return cudaGetLastError();
 }

@@ -728,7 +728,7 @@ struct B3Cfg {
   static constexpr int PS_BYTES = kT * kQB * 2;        // P^T or dS [key][query] for one block = 16 KB
   static constexpr int DQ_BYTES = kQB * DH * 4;        // dQ staging, 2 x [32 queries][dh] fp32 = 32 KB
   static constexpr int BAR_BYTES = 1536;               // barriers, rab tables, TMEM slot
-  static constexpr int SMEM = 2 * KTILE + kQStages * QSTAGE + 2 * PS_BYTES + DQ_BYTES + kQStages * TS_BYTES +
+  static constexpr int SMEM = 2 * KTILE + kQStages * QSTAGE + PS_BYTES + DQ_BYTES + kQStages * TS_BYTES +
                               BAR_BYTES;
   static constexpr uint32_t IDESC_ST = idesc_bf16(128, kQB, false, false);   // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DKV = idesc_bf16(128, DH, false, true);    // P^T dO, dS^T Q
@@ -766,8 +766,7 @@ __global__ void __launch_bounds__(kB3Threads, 1)
   uint8_t* sK = smem;
   uint8_t* sV = sK + C::KTILE;
   uint8_t* sQD = sV + C::KTILE;                    // kQStages x (Q | dO)
-  uint8_t* sPT = sQD + kQStages * C::QSTAGE;        // P^T
-  uint8_t* sDS = sPT + C::PS_BYTES;                 // dS
+  uint8_t* sDS = sQD + kQStages * C::QSTAGE;        // dS
   float* sDQ = reinterpret_cast<float*>(sDS + C::PS_BYTES);   // 2 x dQ staging [32][128]
   uint8_t* sTS = sDS + C::PS_BYTES + C::DQ_BYTES;             // kQStages x times
   uint64_t* bars = reinterpret_cast<uint64_t*>(sTS + kQStages * C::TS_BYTES);
@@ -808,7 +807,7 @@ __global__ void __launch_bounds__(kB3Threads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tD = tmem + 64;
-  auto tQ = [tmem](uint32_t b) { return tmem + 128u + b * 64u; };
+  const uint32_t tQ = tmem + 128, tPT = tmem + 192, tDS = tmem + 224;
   const uint32_t tdV = tmem + 256, tdK = tmem + 384;
 
   if (warp < 4) {
@@ -952,25 +951,26 @@ __global__ void __launch_bounds__(kB3Threads, 1)
             const int st = (int)(gp % kQStages);
             if (m == 1 && !mbar_wait(dkv_free, (items_done & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
             if (!mbar_wait(pds_full, gp & 1, abort_flag, P.status)) { ok = false; break; }
-            if (gp >= 2 && !mbar_wait(&dq_free[b], ((gp - 2) >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            if (gp >= 1 && !mbar_wait(&dq_free[0], (gp - 1) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t q_s = smem_u32(sQD + st * C::QSTAGE), do_s = q_s + C::QTILE;
-            const uint32_t pt_s = smem_u32(sPT), ds_s = smem_u32(sDS);
+            const uint32_t ds_s = smem_u32(sDS);
             const uint32_t acc0 = m > 1 ? 1u : 0u;
+            // A = P^T, dS^T from TMEM (16 queries = 8 packed columns per step)
 #pragma unroll
             for (int k = 0; k < kQB / 16; ++k)
-              mma_ss(tdV, sdesc_kmajor(pt_s + k * 32), sdesc_mnmajor(do_s + k * 2048, kQB * 128), C::IDESC_DKV,
+              mma_ts(tdV, tPT + k * 8, sdesc_mnmajor(do_s + k * 2048, kQB * 128), C::IDESC_DKV,
                      (acc0 || k > 0) ? 1u : 0u);
 #pragma unroll
             for (int k = 0; k < kQB / 16; ++k)
-              mma_ss(tdK, sdesc_kmajor(ds_s + k * 32), sdesc_mnmajor(q_s + k * 2048, kQB * 128), C::IDESC_DKV,
+              mma_ts(tdK, tDS + k * 8, sdesc_mnmajor(q_s + k * 2048, kQB * 128), C::IDESC_DKV,
                      (acc0 || k > 0) ? 1u : 0u);
             mma_commit(&qd_empty[st]);
 #pragma unroll
             for (int k = 0; k < kT / 16; ++k)
-              mma_ss(tQ(b), sdesc_mnmajor(k_s + k * 2048, kT * 128), sdesc_mnmajor(ds_s + k * 2048, kT * 128),
+              mma_ss(tQ, sdesc_mnmajor(k_s + k * 2048, kT * 128), sdesc_mnmajor(ds_s + k * 2048, kT * 128),
                      C::IDESC_DQT, k > 0 ? 1u : 0u);
-            mma_commit(&dq_full[b]);
+            mma_commit(&dq_full[0]);
             mma_commit(ps_free);
           }
         }
@@ -1006,17 +1006,17 @@ __global__ void __launch_bounds__(kB3Threads, 1)
       const int nqb = qblocks(n, item.kt);
       for (int m = 0; m < nqb; ++m) {
         const uint32_t gb = g + m, b = gb & 1;
-        const bool f = !mbar_wait(&dq_full[b], (gb >> 1) & 1, abort_flag, P.status);
+        const bool f = !mbar_wait(&dq_full[0], gb & 1, abort_flag, P.status);
         if (tw == 0) bulk_wait_read0();             // the previous block's reduces have read the staging tile
         if (named_barrier_any(4, 128, f)) { fail = true; break; }
         tc_fence_after();
         uint32_t r0[32], r1[32];
-        tmem_ld32(tQ(b) + lane_off, r0);
-        tmem_ld32(tQ(b) + lane_off + 32, r1);
+        tmem_ld32(tQ + lane_off, r0);
+        tmem_ld32(tQ + lane_off + 32, r1);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dq_free[b]);
+        if (lane == 0) mbar_arrive(&dq_free[0]);
 #pragma unroll
         for (int i = 0; i < 32; ++i) sDQ[i * DH + row] = __uint_as_float(r0[i]) * inv_N;
 #pragma unroll
@@ -1250,14 +1250,17 @@ __global__ void __launch_bounds__(kB3Threads, 1)
         }
         // P^T and dS into the tiles once block gb-1's MMAs have read them
         if (gb >= 1) fail = !mbar_wait(ps_free, (gb - 1) & 1, abort_flag, P.status) || fail;
-        uint8_t* ptb = sPT;
+        tc_fence_after();
+        tmem_st16(tPT + lane_off + wg * 16, pk);
+        tmem_st16(tDS + lane_off + wg * 16, dk);
         uint8_t* dsb = sDS;
 #pragma unroll
         for (int g8 = 0; g8 < 4; ++g8) {
           const uint32_t off = mn_off(row, wg * 32 + g8 * 8, kT * 128);
-          *reinterpret_cast<uint4*>(ptb + off) = make_uint4(pk[4 * g8], pk[4 * g8 + 1], pk[4 * g8 + 2], pk[4 * g8 + 3]);
           *reinterpret_cast<uint4*>(dsb + off) = make_uint4(dk[4 * g8], dk[4 * g8 + 1], dk[4 * g8 + 2], dk[4 * g8 + 3]);
         }
+        tmem_st_wait();
+        tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(pds_full);

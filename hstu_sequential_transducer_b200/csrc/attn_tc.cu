@@ -10,24 +10,26 @@
 // Work items are (sequence, head, 128-row query tile), ordered longest-first
 // by a device-side counting sort (attn_sched) and dealt round-robin to one
 // persistent CTA per SM.  Per CTA:
-//   warp 0      K producer: the Q tile once per item; K tiles (128 keys) with
-//               the keys' timestamps into a three-stage ring, freed as soon as
-//               S = Q K^T has read the tile
+//   warp 0      K producer: the Q tile once per item; K tiles (128 keys) into
+//               a three-stage ring, freed as soon as S = Q K^T has read the
+//               tile, and the keys' timestamps into a six-slot ring of their
+//               own (freed when the activation has used them)
 //   warp 10     V producer: V tiles into a two-stage ring, freed by O += P V
-//   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S
-//               buffers; O += P V with P read from TMEM (A operand in TMEM)
+//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into one of three TMEM
+//               S buffers, two tiles ahead of O += P_{j-2} V_{j-2}, which takes
+//               P from TMEM (A operand in TMEM)
 //   warps 2..9  two warpgroups, one query row per thread; warpgroup b takes
-//               the key tiles of S/P buffer b (every other tile, all 128
-//               columns), so one warpgroup's waits and bucket searches
-//               overlap the other's SiLU work: S from TMEM, bucketed rab
-//               bias, mask, SiLU, P (bf16) into its TMEM P buffer; at the
-//               end of an item, half of O each, times 1/N plus the
-//               candidates' self term
+//               every other key tile (all 128 columns), so one warpgroup's
+//               waits and bucket searches overlap the other's SiLU work: S
+//               from TMEM, bucketed rab bias, mask, SiLU, P (bf16) written
+//               over the first half of the tile's own S buffer; at the end of
+//               an item, half of O each, times 1/N plus the candidates' self
+//               term
 // Both producers read timestamps ahead of their waits and keep the next
 // tiles prefetched into L2, so the rings refill at L2 latency.
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O [256,384), P0 [384,448),
-// P1 [448,512).  A commit arrives only when every earlier MMA of the thread
-// is complete, so once S_{j+2} is signalled the PV of tile j has read P_j.
+// TMEM (512 columns): S/P 0..2 at [128 b, 128 b + 128), O [384, 384 + DH).
+// The MMAs of the one issuing thread run in issue order, so S_{j+3}, issued
+// after P_j V_j, overwrites P_j only once that MMA has read it.
 //
 // The rab bias of one row against one key tile is cheap in the common case:
 // away from the diagonal the position bucket is the last one, and the time
@@ -171,14 +173,15 @@ struct FwdCfg {
   static constexpr int TILE_BYTES = kTile * DH * 2;     // one 128 x DH bf16 tile
   static constexpr int K_STAGES = 3;                    // K tiles (and their timestamps)
   static constexpr int V_STAGES = 2;                    // V tiles
-  static constexpr int TS_BYTES = kTile * 8;            // key timestamps of one K stage
-  static constexpr int SMEM_USED = 1024 + TILE_BYTES * (1 + K_STAGES + V_STAGES) + K_STAGES * TS_BYTES + 1024;
+  static constexpr int TS_BYTES = kTile * 8;            // key timestamps of one tile
+  static constexpr int TS_STAGES = 6;                   // timestamp slots (outlive the K stage)
+  static constexpr int SMEM_USED = 1024 + TILE_BYTES * (1 + K_STAGES + V_STAGES) + TS_STAGES * TS_BYTES + 1024;
   // at least half of the SM's shared memory, so that one CTA (and its 512
   // TMEM columns) is resident per SM
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr uint32_t IDESC_S = idesc_bf16(128, kTile, false, false);
   static constexpr uint32_t IDESC_O = idesc_bf16(128, DH, false, true);
-  static constexpr uint32_t TMEM_COLS = 512;            // S0, S1, O, P0, P1
+  static constexpr uint32_t TMEM_COLS = 512;            // S/P 0..2, O
   static constexpr int THREADS = 352;                   // 11 warps (the V producer is warp 10)
   static constexpr int ACT_WARPS = 8;
   static constexpr int PREFETCH = 4;                    // key tiles kept prefetched into L2
@@ -298,17 +301,17 @@ __global__ void __launch_bounds__(352, 1)
   uint8_t* sK = sQ + C::TILE_BYTES;                      // K_STAGES tiles
   uint8_t* sV = sK + C::K_STAGES * C::TILE_BYTES;        // V_STAGES tiles
   uint8_t* sTS = sV + C::V_STAGES * C::TILE_BYTES;       // K_STAGES x timestamps
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sTS + C::K_STAGES * C::TS_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sTS + C::TS_STAGES * C::TS_BYTES);
   uint64_t* q_full = bars;                   // 1
   uint64_t* q_empty = bars + 1;              // 1
   uint64_t* k_full = bars + 2;               // K_STAGES
   uint64_t* k_empty = k_full + C::K_STAGES;  // K_STAGES: S has read the K tile
-  uint64_t* ts_free = k_empty + C::K_STAGES; // K_STAGES (8 warps): the tile's timestamps are read
-  uint64_t* v_full = ts_free + C::K_STAGES;  // V_STAGES
+  uint64_t* ts_free = k_empty + C::K_STAGES; // TS_STAGES (4 warps): the tile's timestamps are read
+  uint64_t* v_full = ts_free + C::TS_STAGES; // V_STAGES
   uint64_t* v_empty = v_full + C::V_STAGES;  // V_STAGES
-  uint64_t* s_full = v_empty + C::V_STAGES;  // 2
-  uint64_t* p_full = s_full + 2;             // 2
-  uint64_t* o_full = p_full + 2;             // 1
+  uint64_t* s_full = v_empty + C::V_STAGES;  // 3
+  uint64_t* p_full = s_full + 3;             // 3
+  uint64_t* o_full = p_full + 3;             // 1
   uint64_t* o_free = o_full + 1;             // 1
   uint64_t* done_bar = o_free + 1;           // 1
   float* rab_all = reinterpret_cast<float*>(done_bar + 1);   // per warpgroup [2][32] of its head
@@ -325,15 +328,15 @@ __global__ void __launch_bounds__(352, 1)
     for (int s = 0; s < C::K_STAGES; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
-      mbar_init(&ts_free[s], C::ACT_WARPS / 2);      // the warpgroup that took the tile
     }
+    for (int s = 0; s < C::TS_STAGES; ++s) mbar_init(&ts_free[s], C::ACT_WARPS / 2);   // the warpgroup that took the tile
     for (int s = 0; s < C::V_STAGES; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], C::ACT_WARPS / 2);       // the warpgroup of buffer i
+      mbar_init(&p_full[i], C::ACT_WARPS / 2);       // the warpgroup of the tile in buffer i
     }
     mbar_init(o_full, 1);
     mbar_init(o_free, C::ACT_WARPS);
@@ -346,14 +349,18 @@ __global__ void __launch_bounds__(352, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // S buffer b at columns [128 b, 128 b + 128), O at [256, 384), P buffer b at [384 + 64 b, ...)
+  // S buffer b at columns [128 b, 128 b + 128) (b < 3); P of the tile is
+  // written over the first 64 columns of its own S buffer (bf16 pairs), chunk
+  // c over S columns [16 c, 16 c + 16), which chunk c / 2 <= c has already
+  // loaded; O at [384, 384 + DH)
   auto tS = [tmem](uint32_t b) { return tmem + b * 128u; };
-  const uint32_t tO = tmem + 256;
-  auto tP = [tmem](uint32_t b) { return tmem + 384u + b * 64u; };
+  const uint32_t tO = tmem + 384;
+  auto tP = [tmem](uint32_t b) { return tmem + b * 128u; };
 
   // Every role walks the same item sequence and numbers the key tiles it
   // meets with one running counter n: K stage n % K_STAGES (parity
-  // (n / K_STAGES) & 1), V stage n % V_STAGES, S/P buffer n & 1.
+  // (n / K_STAGES) & 1), timestamp slot n % TS_STAGES, V stage n % V_STAGES,
+  // S/P buffer n % 3 (parity (n / 3) & 1); warpgroup n & 1 takes tile n.
   if (warp == 0) {
     // ------------------------------------------------------------ K producer
     uint32_t n = 0, items_done = 0;
@@ -406,13 +413,15 @@ __global__ void __launch_bounds__(352, 1)
           const int c = lane + 32 * q;
           tk[q] = (k0 + c < kend) ? a.kv_ts[g.ks + k0 + c] : (1LL << 62);
         }
+        const int tslot = (int)(n % C::TS_STAGES);
+        const uint32_t tpar = (n / C::TS_STAGES) & 1;
         if (lane == 0) {
           ok = mbar_wait(&k_empty[stage], par ^ 1, abort_flag, P.status);
-          ok = ok && mbar_wait(&ts_free[stage], par ^ 1, abort_flag, P.status);
+          ok = ok && mbar_wait(&ts_free[tslot], tpar ^ 1, abort_flag, P.status);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        long long* kts = reinterpret_cast<long long*>(sTS + stage * C::TS_BYTES);
+        long long* kts = reinterpret_cast<long long*>(sTS + tslot * C::TS_BYTES);
 #pragma unroll
         for (int q = 0; q < 4; ++q) kts[lane + 32 * q] = tk[q];
         __syncwarp();
@@ -488,9 +497,10 @@ __global__ void __launch_bounds__(352, 1)
         tc_fence_after();
         const uint32_t q0 = smem_u32(sQ);
         bool ok = true;
-        for (int j = 0; j <= nk; ++j) {
+        // S runs two tiles ahead of P V: S_j goes to buffer (n + j) % 3, whose
+        // previous tile's P V was issued (and its P read) before
+        for (int j = 0; j <= nk + 1; ++j) {
           if (j < nk) {
-            // S_j = Q K_j^T into buffer (n + j) & 1
             const uint32_t nj = n + j;
             const int stage = (int)(nj % C::K_STAGES);
             if (!mbar_wait(&k_full[stage], (nj / C::K_STAGES) & 1, abort_flag, P.status)) { ok = false; break; }
@@ -499,25 +509,25 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
             for (int k = 0; k < DH / 16; ++k) {
               const uint32_t off = (k / 4) * (kTile * 128) + (k % 4) * 32;
-              mma_ss(tS(nj & 1), sdesc_kmajor(q0 + off), sdesc_kmajor(k0s + off), C::IDESC_S, k > 0);
+              mma_ss(tS(nj % 3), sdesc_kmajor(q0 + off), sdesc_kmajor(k0s + off), C::IDESC_S, k > 0);
             }
-            mma_commit(&s_full[nj & 1]);
+            mma_commit(&s_full[nj % 3]);
             mma_commit(&k_empty[stage]);
             if (j == nk - 1) mma_commit(q_empty);
           }
-          if (j >= 1) {
-            // O += P_{j-1} V_{j-1}
-            const uint32_t np = n + j - 1;
-            if (j == 1 && !mbar_wait(o_free, (items_done & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
+          if (j >= 2) {
+            // O += P_{j-2} V_{j-2}
+            const uint32_t np = n + j - 2;
+            if (j == 2 && !mbar_wait(o_free, (items_done & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
             const int pst = (int)(np % C::V_STAGES);
             if (!mbar_wait(&v_full[pst], (np / C::V_STAGES) & 1, abort_flag, P.status)) { ok = false; break; }
-            if (!mbar_wait(&p_full[np & 1], (np >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+            if (!mbar_wait(&p_full[np % 3], (np / 3) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t v0 = smem_u32(sV + pst * C::TILE_BYTES);
 #pragma unroll
             for (int k = 0; k < kTile / 16; ++k)
-              mma_ts(tO, tP(np & 1) + k * 8, sdesc_mnmajor(v0 + k * 2048, kTile * 128), C::IDESC_O,
-                     (j > 1 || k > 0) ? 1u : 0u);
+              mma_ts(tO, tP(np % 3) + k * 8, sdesc_mnmajor(v0 + k * 2048, kTile * 128), C::IDESC_O,
+                     (j > 2 || k > 0) ? 1u : 0u);
             mma_commit(&v_empty[pst]);
           }
         }
@@ -568,11 +578,11 @@ __global__ void __launch_bounds__(352, 1)
       const float rp_far = rab[a.P - 1];
       for (int j = (int)((n + wg) & 1); j < nk; j += 2) {   // the tiles of buffer wg
         const uint32_t nj = n + j;
-        const uint32_t buf = nj & 1, par = (nj >> 1) & 1;
+        const uint32_t buf = nj % 3, par = (nj / 3) & 1;
         fail = !mbar_wait(&s_full[buf], par, abort_flag, P.status);
         if (named_barrier_any(bid, 128, fail)) { fail = true; break; }
         tc_fence_after();
-        const int kst = (int)(nj % C::K_STAGES);
+        const int kst = (int)(nj % C::TS_STAGES);
         const long long* kts = reinterpret_cast<const long long*>(sTS + kst * C::TS_BYTES);
         const int k0 = j * kTile;
         // fast path: every key of the tile visible, last position bucket,

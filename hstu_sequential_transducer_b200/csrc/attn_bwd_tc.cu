@@ -147,12 +147,6 @@ __device__ __forceinline__ float tanh_fast(float x) {
 
 constexpr int kBThreads = 320;
 
-// SiLU'(x) = sigma(x) (1 + x (1 - sigma(x))) with sigma(x) = (1 + tanh(x/2)) / 2
-__device__ __forceinline__ float silu_grad_fast(float x) {
-  const float h = 0.5f * x;
-  const float t = tanh_fast(h);
-  return 0.5f * (1.f + t + fmaf(-h * t, t, h));
-}
 constexpr int kPrefetch = 4;   // query blocks the backward producer prefetches ahead
 constexpr int kActWarps = 8;
 

@@ -32,6 +32,17 @@ __device__ __forceinline__ float silu_grad_acc(float x) {
   float s = sigmoid_acc(x);
   return s * (1.0f + x * (1.0f - s));
 }
+// SiLU'(x) = sigma(x) (1 + x (1 - sigma(x))) with sigma(x) = (1 + tanh(x/2)) / 2,
+// on the hardware tanh (relative error near 2^-11): for bf16 results.
+__device__ __forceinline__ float silu_grad_fast(float x) {
+  const float h = 0.5f * x;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return 0.5f * (1.f + t + fmaf(-h * t, t, h));
+}
+// SiLU' in the precision the element type T needs.
+template <typename T> __device__ __forceinline__ float silu_grad_t(float x) { return silu_grad_acc(x); }
+template <> __device__ __forceinline__ float silu_grad_t<bf16>(float x) { return silu_grad_fast(x); }
 
 // ---------------------------------------------------------------------------
 // rab^{p,t} buckets (readings: clamped linear position distance; log2 time

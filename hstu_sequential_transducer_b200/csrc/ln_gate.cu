@@ -59,7 +59,8 @@ __device__ __forceinline__ void load_f32(const float* p, float* f) {
 }
 
 // CH = vector chunks per lane (d <= 32 * CH * VEC)
-template <typename T, int CH>
+// AFF: gamma/beta given (otherwise the identity affine, and no registers for it)
+template <typename T, int CH, bool AFF>
 __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, const T* __restrict__ gamma,
                                                           const T* __restrict__ beta,
                                                           const float* __restrict__ o,
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
     const int ch = lane + 32 * c;
 #pragma unroll
     for (int k = 0; k < VN; ++k) { gm[c][k] = 1.f; bt[c][k] = 0.f; }
-    if (ch < nchunk) {
+    if (AFF && ch < nchunk) {
       if (gamma) Vec<T>::load(gamma + ch * VN, gm[c]);
       if (beta) Vec<T>::load(beta + ch * VN, bt[c]);
     }
@@ -85,13 +86,14 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
   const int64_t nw = (int64_t)gridDim.x * (blockDim.x / 32);
   const float inv_d = 1.f / (float)d;
   for (int64_t r = warp; r < rows; r += nw) {
-    float x[CH][VN];
+    float x[CH][VN], uu[CH][VN];
     float s = 0.f;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int ch = lane + 32 * c;
       if (ch < nchunk) {
         load_f32<VN>(o + r * d + ch * VN, x[c]);
+        if (!AFF) Vec<T>::load(g + r * g_stride + ch * VN, uu[c]);   // in flight during the reductions
 #pragma unroll
         for (int k = 0; k < VN; ++k) s += x[c][k];
       } else {
@@ -114,9 +116,10 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
       const int ch = lane + 32 * c;
       if (ch < nchunk) {
         float u[VN], out[VN];
-        Vec<T>::load(g + r * g_stride + ch * VN, u);
+        if (AFF) Vec<T>::load(g + r * g_stride + ch * VN, u);
 #pragma unroll
-        for (int k = 0; k < VN; ++k) out[k] = ((x[c][k] - mu) * rs * gm[c][k] + bt[c][k]) * u[k];
+        for (int k = 0; k < VN; ++k)
+          out[k] = AFF ? ((x[c][k] - mu) * rs * gm[c][k] + bt[c][k]) * u[k] : (x[c][k] - mu) * rs * uu[c][k];
         Vec<T>::store(z + r * d + ch * VN, out);
       }
     }
@@ -127,8 +130,8 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
   }
 }
 
-template <typename T, int CH>
-__global__ void __launch_bounds__(256) ln_gate_bwd_kernel(
+template <typename T, int CH, bool AFF>
+__global__ void __launch_bounds__(256, AFF ? 1 : 2) ln_gate_bwd_kernel(
     int d, const T* __restrict__ gamma, const T* __restrict__ beta, const T* __restrict__ dz,
     const float* __restrict__ o, const T* __restrict__ g, const T* __restrict__ pre, int64_t g_stride,
     const float* __restrict__ mean, const float* __restrict__ rstd, int64_t rows,
@@ -144,13 +147,15 @@ __global__ void __launch_bounds__(256) ln_gate_bwd_kernel(
     const int ch = lane + 32 * c;
 #pragma unroll
     for (int k = 0; k < VN; ++k) { gm[c][k] = 1.f; bt[c][k] = 0.f; accg[c][k] = 0.f; accb[c][k] = 0.f; }
-    if (ch < nchunk) {
+    if (AFF && ch < nchunk) {
       if (gamma) Vec<T>::load(gamma + ch * VN, gm[c]);
       if (beta) Vec<T>::load(beta + ch * VN, bt[c]);
     }
   }
-  for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) red[i] = 0.f;
-  __syncthreads();
+  if (AFF) {
+    for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) red[i] = 0.f;
+    __syncthreads();
+  }
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int64_t nw = (int64_t)gridDim.x * (blockDim.x / 32);
   const float inv_d = 1.f / (float)d;
@@ -170,12 +175,14 @@ __global__ void __launch_bounds__(256) ln_gate_bwd_kernel(
 #pragma unroll
         for (int k = 0; k < VN; ++k) {
           oh[c][k] = (x[k] - mu) * rs;
-          const float ln = oh[c][k] * gm[c][k] + bt[c][k];
+          const float ln = AFF ? oh[c][k] * gm[c][k] + bt[c][k] : oh[c][k];
           const float dln = gz[k] * u[k];
-          du[k] = gz[k] * ln * silu_grad_acc(pu[k]);
-          accg[c][k] += dln * oh[c][k];
-          accb[c][k] += dln;
-          dh[c][k] = dln * gm[c][k];
+          du[k] = gz[k] * ln * silu_grad_t<T>(pu[k]);
+          if (AFF) {
+            accg[c][k] += dln * oh[c][k];
+            accb[c][k] += dln;
+          }
+          dh[c][k] = AFF ? dln * gm[c][k] : dln;
           sa += dh[c][k];
           sb += dh[c][k] * oh[c][k];
         }
@@ -198,7 +205,7 @@ __global__ void __launch_bounds__(256) ln_gate_bwd_kernel(
       }
     }
   }
-  if (dgamma || dbeta) {
+  if (AFF && (dgamma || dbeta)) {
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int ch = lane + 32 * c;
@@ -228,7 +235,7 @@ int num_sms() {
   return n;
 }
 
-template <typename T, int CH>
+template <typename T, int CH, bool AFF>
 cudaError_t fwd_ch(int d, float eps, const void* gamma, const void* beta, const float* o,
                    const void* g, int64_t gs, int64_t T_, void* z, float* mean, float* rstd,
                    cudaStream_t s) {
@@ -236,13 +243,13 @@ cudaError_t fwd_ch(int d, float eps, const void* gamma, const void* beta, const 
   const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
   if (blocks == 0) return cudaSuccess;
-  ln_gate_fwd_kernel<T, CH><<<(unsigned)blocks, 256, 0, s>>>(
+  ln_gate_fwd_kernel<T, CH, AFF><<<(unsigned)blocks, 256, 0, s>>>(
       d, eps, (const T*)gamma, (const T*)beta, o, (const T*)g, gs, T_, (T*)z, mean, rstd);
   count_launch();
   return cudaGetLastError();
 }
 
-template <typename T, int CH>
+template <typename T, int CH, bool AFF>
 cudaError_t bwd_ch(int d, const void* gamma, const void* beta, const void* dz, const float* o,
                    const void* g, const void* pre, int64_t gs, const float* mean, const float* rstd,
                    int64_t T_, void* dout, void* dpre, float* dgamma, float* dbeta, cudaStream_t s) {
@@ -250,7 +257,7 @@ cudaError_t bwd_ch(int d, const void* gamma, const void* beta, const void* dz, c
   const int64_t cap = (int64_t)num_sms() * 4;
   if (blocks > cap) blocks = cap;
   if (blocks == 0) return cudaSuccess;
-  ln_gate_bwd_kernel<T, CH><<<(unsigned)blocks, 256, 2 * d * sizeof(float), s>>>(
+  ln_gate_bwd_kernel<T, CH, AFF><<<(unsigned)blocks, 256, AFF ? 2 * d * sizeof(float) : 0, s>>>(
       d, (const T*)gamma, (const T*)beta, (const T*)dz, o, (const T*)g, (const T*)pre, gs,
       mean, rstd, T_, (T*)dout, (T*)dpre, dgamma, dbeta);
   count_launch();
@@ -264,16 +271,25 @@ cudaError_t ln_gate_fwd(int dtype, int d, float eps, const void* gamma, const vo
                         float* rstd, cudaStream_t s) {
   const int vn = dtype == HSTU_BF16 ? 8 : 4;
   const int ch = (d / vn + 31) / 32;
+  const bool aff = gamma || beta;
   if (dtype == HSTU_BF16) {
-    if (ch <= 1) return fwd_ch<bf16, 1>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
-    if (ch <= 2) return fwd_ch<bf16, 2>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
-    if (ch <= 4) return fwd_ch<bf16, 4>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
-    if (ch <= 8) return fwd_ch<bf16, 8>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
+    if (ch <= 1) return aff ? fwd_ch<bf16, 1, true>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s)
+                        : fwd_ch<bf16, 1, false>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
+    if (ch <= 2) return aff ? fwd_ch<bf16, 2, true>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s)
+                        : fwd_ch<bf16, 2, false>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
+    if (ch <= 4) return aff ? fwd_ch<bf16, 4, true>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s)
+                        : fwd_ch<bf16, 4, false>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
+    if (ch <= 8) return aff ? fwd_ch<bf16, 8, true>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s)
+                        : fwd_ch<bf16, 8, false>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
   } else {
-    if (ch <= 1) return fwd_ch<float, 1>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
-    if (ch <= 2) return fwd_ch<float, 2>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
-    if (ch <= 4) return fwd_ch<float, 4>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
-    if (ch <= 8) return fwd_ch<float, 8>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
+    if (ch <= 1) return aff ? fwd_ch<float, 1, true>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s)
+                        : fwd_ch<float, 1, false>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
+    if (ch <= 2) return aff ? fwd_ch<float, 2, true>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s)
+                        : fwd_ch<float, 2, false>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
+    if (ch <= 4) return aff ? fwd_ch<float, 4, true>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s)
+                        : fwd_ch<float, 4, false>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
+    if (ch <= 8) return aff ? fwd_ch<float, 8, true>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s)
+                        : fwd_ch<float, 8, false>(d, eps, gamma, beta, o, g, gs, T_, z, mean, rstd, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -284,8 +300,12 @@ cudaError_t ln_gate_bwd(int dtype, int d, const void* gamma, const void* beta, c
                         float* dgamma, float* dbeta, cudaStream_t s) {
   const int vn = dtype == HSTU_BF16 ? 8 : 4;
   const int ch = (d / vn + 31) / 32;
-#define HSTU_LNB(TT, C) \
-  return bwd_ch<TT, C>(d, gamma, beta, dz, o, g, pre, gs, mean, rstd, T_, dout, dpre, dgamma, dbeta, s)
+  const bool aff = gamma || beta || dgamma || dbeta;
+#define HSTU_LNB(TT, C)                                                                                     \
+  return aff ? bwd_ch<TT, C, true>(d, gamma, beta, dz, o, g, pre, gs, mean, rstd, T_, dout, dpre, dgamma,  \
+                                   dbeta, s)                                                                \
+             : bwd_ch<TT, C, false>(d, gamma, beta, dz, o, g, pre, gs, mean, rstd, T_, dout, dpre, dgamma, \
+                                    dbeta, s)
   if (dtype == HSTU_BF16) {
     if (ch <= 1) HSTU_LNB(bf16, 1);
     if (ch <= 2) HSTU_LNB(bf16, 2);

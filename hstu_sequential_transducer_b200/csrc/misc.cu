@@ -40,6 +40,33 @@ __global__ void dq_finalize_kernel(const float* __restrict__ dq, const T* __rest
   }
 }
 
+// bf16, d and the Pre stride multiples of 8, 16-byte aligned rows: eight
+// columns per thread and step (two fp32 vectors of dQ, one bf16 vector of Pre)
+__global__ void dq_finalize_bf16x8_kernel(const float* __restrict__ dq, const bf16* __restrict__ pre_q,
+                                          int64_t pre_stride, bf16* __restrict__ dpre_q, int64_t rows,
+                                          int d) {
+  const int dv = d / 8;
+  const int64_t n = rows * dv;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / dv;
+    const int c = (int)(i - r * dv) * 8;
+    const float4 a = *reinterpret_cast<const float4*>(dq + r * d + c);
+    const float4 b = *reinterpret_cast<const float4*>(dq + r * d + c + 4);
+    const uint4 pu = *reinterpret_cast<const uint4*>(pre_q + r * pre_stride + c);
+    const __nv_bfloat162* ph = reinterpret_cast<const __nv_bfloat162*>(&pu);
+    const float g[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint4 o;
+    __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 pf = __bfloat1622float2(ph[k]);
+      oh[k] = __floats2bfloat162_rn(g[2 * k] * silu_grad_fast(pf.x), g[2 * k + 1] * silu_grad_fast(pf.y));
+    }
+    *reinterpret_cast<uint4*>(dpre_q + r * pre_stride + c) = o;
+  }
+}
+
 template <typename T>
 __global__ void copy_columns_kernel(const T* __restrict__ src, int64_t ss, T* __restrict__ dst,
                                     int64_t ds, int64_t rows, int64_t cols) {
@@ -130,7 +157,12 @@ cudaError_t dq_finalize(int dtype, const float* dq, const void* pre_q, int64_t p
                         int64_t T, int d, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const unsigned g = grid_for(T * d, 256);
-  if (dtype == HSTU_BF16)
+  const bool vec = d % 8 == 0 && ps % 8 == 0 && ((uintptr_t)dq & 15) == 0 && ((uintptr_t)pre_q & 15) == 0 &&
+                   ((uintptr_t)dpre_q & 15) == 0;
+  if (dtype == HSTU_BF16 && vec)
+    dq_finalize_bf16x8_kernel<<<grid_for(T * (d / 8), 256), 256, 0, s>>>(dq, (const bf16*)pre_q, ps,
+                                                                        (bf16*)dpre_q, T, d);
+  else if (dtype == HSTU_BF16)
     dq_finalize_kernel<bf16><<<g, 256, 0, s>>>(dq, (const bf16*)pre_q, ps, (bf16*)dpre_q, T, d);
   else
     dq_finalize_kernel<float><<<g, 256, 0, s>>>(dq, (const float*)pre_q, ps, (float*)dpre_q, T, d);

@@ -1124,7 +1124,7 @@ __global__ void __launch_bounds__(kB3Threads, 1)
           b_lo = tb64(qts[wg * 32] - tk, a.Bt);
           nb = tb64(qts[wg * 32 + 31] - tk, a.Bt) - b_lo;
         }
-        const bool fast = __all_sync(0xffffffffu, full && far && nb <= 2);
+        const bool fast = __all_sync(0xffffffffu, full && far && nb <= 1);
         // off the fast path: a warp with no allowed pair in its 32 columns
         // writes zeros; gaps within +-2^31 s take 32-bit bucket arithmetic
         const int lastc = min(31, n - 1 - qf);
@@ -1163,8 +1163,7 @@ __global__ void __launch_bounds__(kB3Threads, 1)
           constexpr int E0 = decltype(e0c)::value;
           if (fast) {
             if (nbw == 0) bwd_chunk_fast<0, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
-            else if (nbw == 1) bwd_chunk_fast<1, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
-            else bwd_chunk_fast<2, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
+            else bwd_chunk_fast<1, E0, 16>(sr, dr, 0, hb, p, hd, pk, dk, tot, suf);
             return;
           }
           if (!anyok) {

@@ -244,6 +244,15 @@ __device__ __forceinline__ void bwd_chunk_fast(const uint32_t (&sr)[32], const u
   }
 }
 
+// Shared-memory float reduction issued only where pred holds (a predicated
+// instruction, so per-element bucket sums need no divergent branch).
+__device__ __forceinline__ void pred_red(float* addr, float v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t@p red.shared.add.f32 [%0], %1;\n\t}" ::"r"(smem_u32(addr)),
+      "f"(v), "r"((int)pred)
+      : "memory");
+}
+
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
                "f"(d)
@@ -1188,11 +1197,16 @@ __global__ void __launch_bounds__(kB3Threads, 1)
                 const float sg = fmaf(t, 0.5f, 0.5f);
                 const float pa = ok ? fmaf(h, t, h) : 0.f;
                 const float ds = ok ? __uint_as_float(dr[e + u]) * fmaf(sg, fmaf(-h, t, h), sg) : 0.f;
-                if (ok) {
-                  if (bp < a.P - 1) atomicAdd(&drabw[bp], ds);
-                  else far_sum += ds;
-                  add_t(bt, ds);
-                }
+                // bucket sums without branches: the position bucket straight
+                // to shared memory, the time bucket run-length encoded
+                const bool near = ok && bp < a.P - 1;
+                pred_red(&drabw[bp], ds, near);
+                far_sum += (ok && !near) ? ds : 0.f;
+                const int bte = ok ? bt : tb_cur;
+                const bool chg = bte != tb_cur;
+                pred_red(&drabw[32 + max(tb_cur, 0)], t_sum, chg && tb_cur >= 0);
+                t_sum = chg ? ds : t_sum + ds;
+                tb_cur = bte;
                 pv[u] = pa;
                 dv[u] = ds;
               }

@@ -706,10 +706,10 @@ int sms();
 // registers.  A warpgroup of its own drains dQ^T(g) (transposes it into a
 // dense fp32 tile in shared memory and adds it to the fp32 dQ accumulator
 // with TMA bulk reduce-adds; rows past the sequence end carry exact zeros),
-// so the activation warps go from one block to the next without it; they
-// also finish an item with dK, dV times SiLU'(Pre) into dPre, with the Pre
-// loads in flight during the TMEM loads, while the producer has the next
-// item's K and V tiles prefetched into L2.  Off the fast path, a warp whose 32
+// so the activation warps go from one block to the next without it; the
+// same warpgroup finishes an item with dK, dV times SiLU'(Pre) into dPre
+// while the activation warps already work on the next item, whose K and V
+// tiles the producer has prefetched into L2.  Off the fast path, a warp whose 32
 // columns hold no allowed pair writes zeros, and time gaps within +-2^31 s
 // take 32-bit bucket arithmetic.  Q/dO blocks come through a
 // three-stage ring that the producer keeps prefetched into L2, so block g+1's
@@ -743,10 +743,10 @@ __device__ __forceinline__ int qblocks(int n, int kt) { return (n - kt * kT + kQ
 
 // Warp roles of the dh = 128 kernel: warpgroup 0 = producer (warp 0), MMA
 // issuer (warp 1), two idle warps; warpgroups 1 and 2 = key-row warps;
-// warpgroup 3 = dQ drain.  The 65,536 registers of the launch (512 threads x
-// 128) are re-split with setmaxnreg: 9,216 + 2 x 22,528 + 10,240.
+// warpgroup 3 = dQ drain and the item's dK, dV epilogue.  The 65,536 registers of the launch (512 threads x
+// 128) are re-split with setmaxnreg: 9,216 + 2 x 21,504 + 12,288.
 constexpr int kB3Threads = 512;
-constexpr int kRegCtl = 72, kRegAct = 176, kRegDrain = 80;
+constexpr int kRegCtl = 72, kRegAct = 168, kRegDrain = 96;
 static_assert(128 * (kRegCtl + 2 * kRegAct + kRegDrain) <= 65536, "register split");
 template <int R>
 __device__ __forceinline__ void reg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R)); }
@@ -797,8 +797,8 @@ __global__ void __launch_bounds__(kB3Threads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 22; ++i) {
-      const bool act = (i == 7 || i == 8 || i == 9 || i == 17);
-      const bool drn = (i == 14 || i == 15);
+      const bool act = (i == 7 || i == 8 || i == 9);
+      const bool drn = (i == 14 || i == 15 || i == 17);
       mbar_init(&bars[i], act ? kActWarps : drn ? 4 : 1);
     }
     *abort_flag = 0;
@@ -998,7 +998,7 @@ __global__ void __launch_bounds__(kB3Threads, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int tw = threadIdx.x & 127;
     const float inv_N = a.inv_N;
-    uint32_t g = 0;
+    uint32_t g = 0, items_done = 0;
     bool fail = false;
     for (int it = blockIdx.x; it < total && !fail; it += gridDim.x) {
       const BItem item = P.w.items[it];
@@ -1033,7 +1033,60 @@ __global__ void __launch_bounds__(kB3Threads, 1)
           bulk_commit();
         }
       }
+      if (fail) break;
       g += nqb;
+      // the item's dK, dV times 1/N and SiLU'(Pre) into dPre: this thread's
+      // key row, 16 columns of each at a time
+      if (!mbar_wait(dkv_full, items_done & 1, abort_flag, P.status)) { fail = true; break; }
+      ++items_done;
+      tc_fence_after();
+      {
+        const int jk = k0 + row;
+        const bool kvalid = jk < hlen;
+        const bf16* pre = static_cast<const bf16*>(P.A.pre);
+        bf16* dpre = static_cast<bf16*>(P.A.dpre);
+        const int d = P.A.d;
+        const int64_t rowoff = (s0 + jk) * P.A.pre_stride;
+#pragma unroll 1
+        for (int c = 0; c < DH / 16; ++c) {
+          uint32_t rv[16], rk[16];
+          tmem_ld16(tdV + lane_off + c * 16, rv);
+          tmem_ld16(tdK + lane_off + c * 16, rk);
+          const int col = item.h * DH + c * 16;
+          uint4 pv4[2], pk4[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            pv4[i] = kvalid ? *reinterpret_cast<const uint4*>(pre + rowoff + d + col + 8 * i) : make_uint4(0, 0, 0, 0);
+            pk4[i] = kvalid ? *reinterpret_cast<const uint4*>(pre + rowoff + 3 * d + col + 8 * i) : make_uint4(0, 0, 0, 0);
+          }
+          tmem_ld_wait();
+          if (kvalid) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const __nv_bfloat162* pvh = reinterpret_cast<const __nv_bfloat162*>(&pv4[i]);
+              const __nv_bfloat162* pkh = reinterpret_cast<const __nv_bfloat162*>(&pk4[i]);
+              uint4 ov, ok4;
+              uint32_t* ovw = reinterpret_cast<uint32_t*>(&ov);
+              uint32_t* okw = reinterpret_cast<uint32_t*>(&ok4);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 fv = __bfloat1622float2(pvh[u]);
+                const float2 fk = __bfloat1622float2(pkh[u]);
+                const int j = 8 * i + 2 * u;
+                ovw[u] = pack_bf16(__uint_as_float(rv[j]) * inv_N * silu_grad_fast(fv.x),
+                                   __uint_as_float(rv[j + 1]) * inv_N * silu_grad_fast(fv.y));
+                okw[u] = pack_bf16(__uint_as_float(rk[j]) * inv_N * silu_grad_fast(fk.x),
+                                   __uint_as_float(rk[j + 1]) * inv_N * silu_grad_fast(fk.y));
+              }
+              *reinterpret_cast<uint4*>(dpre + rowoff + d + col + 8 * i) = ov;
+              *reinterpret_cast<uint4*>(dpre + rowoff + 3 * d + col + 8 * i) = ok4;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dkv_free);
     }
     if (tw == 0) bulk_wait0();
   } else {
@@ -1282,54 +1335,6 @@ __global__ void __launch_bounds__(kB3Threads, 1)
       for (int o = 16; o > 0; o >>= 1) far_sum += __shfl_xor_sync(0xffffffffu, far_sum, o);
       if (lane == 0 && far_sum != 0.f) atomicAdd(&drabw[a.P - 1], far_sum);
       g += nqb;
-      // this warpgroup's half of dK, dV (times 1/N and SiLU'(Pre)) into dPre
-      fail = !mbar_wait(dkv_full, items_done & 1, abort_flag, P.status) || fail;
-      ++items_done;
-      if (named_barrier_any(bid, 128, fail)) { fail = true; break; }
-      tc_fence_after();
-      const bf16* pre = static_cast<const bf16*>(P.A.pre);
-      bf16* dpre = static_cast<bf16*>(P.A.dpre);
-      const int64_t rowoff = (s0 + jk) * P.A.pre_stride;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = wg * 2 + cc;
-        uint32_t rv[32], rk[32];
-        tmem_ld32(tdV + lane_off + c * 32, rv);
-        tmem_ld32(tdK + lane_off + c * 32, rk);
-        const int col = item.h * DH + c * 32;
-        uint4 pv4[4], pk4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          pv4[i] = kvalid ? *reinterpret_cast<const uint4*>(pre + rowoff + d + col + 8 * i) : make_uint4(0, 0, 0, 0);
-          pk4[i] = kvalid ? *reinterpret_cast<const uint4*>(pre + rowoff + 3 * d + col + 8 * i) : make_uint4(0, 0, 0, 0);
-        }
-        tmem_ld_wait();
-        if (kvalid) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162* pvh = reinterpret_cast<const __nv_bfloat162*>(&pv4[i]);
-            const __nv_bfloat162* pkh = reinterpret_cast<const __nv_bfloat162*>(&pk4[i]);
-            uint4 ov, ok4;
-            uint32_t* ovw = reinterpret_cast<uint32_t*>(&ov);
-            uint32_t* okw = reinterpret_cast<uint32_t*>(&ok4);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 fv = __bfloat1622float2(pvh[u]);
-              const float2 fk = __bfloat1622float2(pkh[u]);
-              const int j = 8 * i + 2 * u;
-              ovw[u] = pack_bf16(__uint_as_float(rv[j]) * inv_N * silu_grad_fast(fv.x),
-                                 __uint_as_float(rv[j + 1]) * inv_N * silu_grad_fast(fv.y));
-              okw[u] = pack_bf16(__uint_as_float(rk[j]) * inv_N * silu_grad_fast(fk.x),
-                                 __uint_as_float(rk[j + 1]) * inv_N * silu_grad_fast(fk.y));
-            }
-            *reinterpret_cast<uint4*>(dpre + rowoff + d + col + 8 * i) = ov;
-            *reinterpret_cast<uint4*>(dpre + rowoff + 3 * d + col + 8 * i) = ok4;
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dkv_free);
     }
     // flush the last head's bucket sums
     named_barrier(bid, 128);

@@ -130,34 +130,35 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
   }
 }
 
+// AFF: gamma/beta and their gradients live in shared memory (gamma, beta
+// once per CTA; dgamma/dbeta partials per warp, each lane updating only the
+// columns it owns, so no atomics until the CTA's final flush), which keeps the
+// kernel at two CTAs per SM.  Dynamic shared memory: (2 + 2 * warps) * d floats.
 template <typename T, int CH, bool AFF>
-__global__ void __launch_bounds__(256, AFF ? 1 : 2) ln_gate_bwd_kernel(
+__global__ void __launch_bounds__(256, CH <= 4 ? 2 : 1) ln_gate_bwd_kernel(
     int d, const T* __restrict__ gamma, const T* __restrict__ beta, const T* __restrict__ dz,
     const float* __restrict__ o, const T* __restrict__ g, const T* __restrict__ pre, int64_t g_stride,
     const float* __restrict__ mean, const float* __restrict__ rstd, int64_t rows,
     T* __restrict__ dout, T* __restrict__ dpre, float* __restrict__ dgamma,
     float* __restrict__ dbeta) {
   constexpr int VN = Vec<T>::N;
-  extern __shared__ float red[];  // [2][d]
-  const int lane = threadIdx.x % 32;
+  extern __shared__ __align__(16) float sh[];   // gm[d], bt[d], then [warps][2][d] partials
+  const int lane = threadIdx.x % 32, wid = threadIdx.x / 32;
+  const int nwarps = blockDim.x / 32;
   const int nchunk = d / VN;
-  float gm[CH][VN], bt[CH][VN], accg[CH][VN], accb[CH][VN];
-#pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int ch = lane + 32 * c;
-#pragma unroll
-    for (int k = 0; k < VN; ++k) { gm[c][k] = 1.f; bt[c][k] = 0.f; accg[c][k] = 0.f; accb[c][k] = 0.f; }
-    if (AFF && ch < nchunk) {
-      if (gamma) Vec<T>::load(gamma + ch * VN, gm[c]);
-      if (beta) Vec<T>::load(beta + ch * VN, bt[c]);
-    }
-  }
+  float* const sgm = sh;
+  float* const sbt = sh + d;
+  float* const sacc = sh + 2 * d + wid * 2 * d;       // this warp's dgamma, dbeta partials
   if (AFF) {
-    for (int i = threadIdx.x; i < 2 * d; i += blockDim.x) red[i] = 0.f;
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+      sgm[i] = gamma ? to_f(gamma[i]) : 1.f;
+      sbt[i] = beta ? to_f(beta[i]) : 0.f;
+    }
+    for (int i = threadIdx.x; i < 2 * d * nwarps; i += blockDim.x) sh[2 * d + i] = 0.f;
     __syncthreads();
   }
-  const int64_t warp = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  const int64_t nw = (int64_t)gridDim.x * (blockDim.x / 32);
+  const int64_t warp = (int64_t)blockIdx.x * nwarps + wid;
+  const int64_t nw = (int64_t)gridDim.x * nwarps;
   const float inv_d = 1.f / (float)d;
   for (int64_t r = warp; r < rows; r += nw) {
     const float mu = mean[r], rs = rstd[r];
@@ -172,19 +173,33 @@ __global__ void __launch_bounds__(256, AFF ? 1 : 2) ln_gate_bwd_kernel(
         Vec<T>::load(dz + r * d + ch * VN, gz);
         Vec<T>::load(g + r * g_stride + ch * VN, u);
         Vec<T>::load(pre + r * g_stride + ch * VN, pu);
+        float gm[VN], bt[VN], ag[VN], ab[VN];
+        if (AFF) {
+          load_f32<VN>(sgm + ch * VN, gm);
+          load_f32<VN>(sbt + ch * VN, bt);
+          load_f32<VN>(sacc + ch * VN, ag);
+          load_f32<VN>(sacc + d + ch * VN, ab);
+        }
 #pragma unroll
         for (int k = 0; k < VN; ++k) {
           oh[c][k] = (x[k] - mu) * rs;
-          const float ln = AFF ? oh[c][k] * gm[c][k] + bt[c][k] : oh[c][k];
+          const float ln = AFF ? oh[c][k] * gm[k] + bt[k] : oh[c][k];
           const float dln = gz[k] * u[k];
           du[k] = gz[k] * ln * silu_grad_t<T>(pu[k]);
           if (AFF) {
-            accg[c][k] += dln * oh[c][k];
-            accb[c][k] += dln;
+            ag[k] += dln * oh[c][k];
+            ab[k] += dln;
           }
-          dh[c][k] = AFF ? dln * gm[c][k] : dln;
+          dh[c][k] = AFF ? dln * gm[k] : dln;
           sa += dh[c][k];
           sb += dh[c][k] * oh[c][k];
+        }
+        if (AFF) {
+#pragma unroll
+          for (int k = 0; k < VN; k += 4) {
+            *reinterpret_cast<float4*>(sacc + ch * VN + k) = make_float4(ag[k], ag[k + 1], ag[k + 2], ag[k + 3]);
+            *reinterpret_cast<float4*>(sacc + d + ch * VN + k) = make_float4(ab[k], ab[k + 1], ab[k + 2], ab[k + 3]);
+          }
         }
         Vec<T>::store(dpre + r * g_stride + ch * VN, du);
       } else {
@@ -206,20 +221,15 @@ __global__ void __launch_bounds__(256, AFF ? 1 : 2) ln_gate_bwd_kernel(
     }
   }
   if (AFF && (dgamma || dbeta)) {
-#pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      const int ch = lane + 32 * c;
-      if (ch < nchunk)
-#pragma unroll
-        for (int k = 0; k < VN; ++k) {
-          atomicAdd(&red[ch * VN + k], accg[c][k]);
-          atomicAdd(&red[d + ch * VN + k], accb[c][k]);
-        }
-    }
     __syncthreads();
     for (int i = threadIdx.x; i < d; i += blockDim.x) {
-      if (dgamma) atomicAdd(dgamma + i, red[i]);
-      if (dbeta) atomicAdd(dbeta + i, red[d + i]);
+      float vg = 0.f, vb = 0.f;
+      for (int w = 0; w < nwarps; ++w) {
+        vg += sh[2 * d + w * 2 * d + i];
+        vb += sh[2 * d + w * 2 * d + d + i];
+      }
+      if (dgamma) atomicAdd(dgamma + i, vg);
+      if (dbeta) atomicAdd(dbeta + i, vb);
     }
   }
 }
@@ -257,7 +267,13 @@ cudaError_t bwd_ch(int d, const void* gamma, const void* beta, const void* dz, c
   const int64_t cap = (int64_t)num_sms() * 4;
   if (blocks > cap) blocks = cap;
   if (blocks == 0) return cudaSuccess;
-  ln_gate_bwd_kernel<T, CH, AFF><<<(unsigned)blocks, 256, AFF ? 2 * d * sizeof(float) : 0, s>>>(
+  const size_t smem = AFF ? (size_t)(2 + 2 * 8) * d * sizeof(float) : 0;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(ln_gate_bwd_kernel<T, CH, AFF>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  ln_gate_bwd_kernel<T, CH, AFF><<<(unsigned)blocks, 256, smem, s>>>(
       d, (const T*)gamma, (const T*)beta, (const T*)dz, o, (const T*)g, (const T*)pre, gs,
       mean, rstd, T_, (T*)dout, (T*)dpre, dgamma, dbeta);
   count_launch();

@@ -59,7 +59,8 @@ __device__ __forceinline__ void load_f32(const float* p, float* f) {
 }
 
 // CH = vector chunks per lane (d <= 32 * CH * VEC)
-// AFF: gamma/beta given (otherwise the identity affine, and no registers for it)
+// AFF: gamma/beta given, kept in shared memory (dynamic, 2 * d floats);
+// otherwise the identity affine
 template <typename T, int CH, bool AFF>
 __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, const T* __restrict__ gamma,
                                                           const T* __restrict__ beta,
@@ -69,18 +70,15 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
                                                           float* __restrict__ mean_out,
                                                           float* __restrict__ rstd_out) {
   constexpr int VN = Vec<T>::N;
+  extern __shared__ __align__(16) float shf[];     // gm[d], bt[d]
   const int lane = threadIdx.x % 32;
   const int nchunk = d / VN;
-  float gm[CH][VN], bt[CH][VN];
-#pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int ch = lane + 32 * c;
-#pragma unroll
-    for (int k = 0; k < VN; ++k) { gm[c][k] = 1.f; bt[c][k] = 0.f; }
-    if (AFF && ch < nchunk) {
-      if (gamma) Vec<T>::load(gamma + ch * VN, gm[c]);
-      if (beta) Vec<T>::load(beta + ch * VN, bt[c]);
+  if (AFF) {
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+      shf[i] = gamma ? to_f(gamma[i]) : 1.f;
+      shf[d + i] = beta ? to_f(beta[i]) : 0.f;
     }
+    __syncthreads();
   }
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int64_t nw = (int64_t)gridDim.x * (blockDim.x / 32);
@@ -93,7 +91,7 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
       const int ch = lane + 32 * c;
       if (ch < nchunk) {
         load_f32<VN>(o + r * d + ch * VN, x[c]);
-        if (!AFF) Vec<T>::load(g + r * g_stride + ch * VN, uu[c]);   // in flight during the reductions
+        Vec<T>::load(g + r * g_stride + ch * VN, uu[c]);   // in flight during the reductions
 #pragma unroll
         for (int k = 0; k < VN; ++k) s += x[c][k];
       } else {
@@ -115,11 +113,14 @@ __global__ void __launch_bounds__(256) ln_gate_fwd_kernel(int d, float eps, cons
     for (int c = 0; c < CH; ++c) {
       const int ch = lane + 32 * c;
       if (ch < nchunk) {
-        float u[VN], out[VN];
-        if (AFF) Vec<T>::load(g + r * g_stride + ch * VN, u);
+        float out[VN], gm[VN], bt[VN];
+        if (AFF) {
+          load_f32<VN>(shf + ch * VN, gm);
+          load_f32<VN>(shf + d + ch * VN, bt);
+        }
 #pragma unroll
         for (int k = 0; k < VN; ++k)
-          out[k] = AFF ? ((x[c][k] - mu) * rs * gm[c][k] + bt[c][k]) * u[k] : (x[c][k] - mu) * rs * uu[c][k];
+          out[k] = AFF ? ((x[c][k] - mu) * rs * gm[k] + bt[k]) * uu[c][k] : (x[c][k] - mu) * rs * uu[c][k];
         Vec<T>::store(z + r * d + ch * VN, out);
       }
     }
@@ -253,7 +254,7 @@ cudaError_t fwd_ch(int d, float eps, const void* gamma, const void* beta, const 
   const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
   if (blocks == 0) return cudaSuccess;
-  ln_gate_fwd_kernel<T, CH, AFF><<<(unsigned)blocks, 256, 0, s>>>(
+  ln_gate_fwd_kernel<T, CH, AFF><<<(unsigned)blocks, 256, AFF ? 2 * d * sizeof(float) : 0, s>>>(
       d, eps, (const T*)gamma, (const T*)beta, o, (const T*)g, gs, T_, (T*)z, mean, rstd);
   count_launch();
   return cudaGetLastError();

@@ -18,6 +18,13 @@
 //               (one staging tile per warpgroup), TMA store (or TMA reduce-add
 //               for split-K); a warpgroup waits for its previous store only
 //               when it next needs its staging tile
+// PAIR: a cluster of two CTAs computes 256-row tiles with tcgen05 cta_group::2:
+// each CTA loads its own 128 rows of A and half of the tile's B columns, the
+// even CTA's MMA thread issues M = 256 MMAs over both SMs' shared memory and
+// TMEM (each CTA holds the accumulator rows of its A rows), its commits arrive
+// on both CTAs' barriers, and both CTAs' loads and epilogues report to the
+// even CTA's barriers.  Per SM this halves the B operand's shared-memory
+// reads and the TMA traffic of B.  No load multicasts.
 // Every mbarrier wait is bounded; a timeout sets the library's device status
 // word and the CTA drains its own copies and MMAs, frees its TMEM and exits.
 #include <cuda.h>
@@ -36,10 +43,10 @@ constexpr int BK = 64;
 constexpr int kThreads = 320;
 constexpr int kMaxSmem = 232448;
 
-template <int BN, bool AK, bool BKM, int EPI, typename TOUT>
+template <int BN, bool AK, bool BKM, int EPI, typename TOUT, bool PAIR>
 struct Cfg {
   static constexpr int A_BYTES = BM * 128;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * 128;   // this CTA's part of the B tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NOUT = EPI == EPI_SILU_SPLIT ? 2 : 1;
   static constexpr int OUT_ES = (int)sizeof(TOUT);
@@ -49,7 +56,7 @@ struct Cfg {
   static constexpr int STAGES_FIT = (kMaxSmem - 1024 - 2 * NOUT * STG_BYTES - BAR_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static constexpr int SMEM = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 2 * NOUT * STG_BYTES + BAR_BYTES;
-  static constexpr uint32_t IDESC = idesc_bf16(BM, BN, !AK, !BKM);
+  static constexpr uint32_t IDESC = idesc_bf16(PAIR ? 2 * BM : BM, BN, !AK, !BKM);
   static_assert(STAGES >= 2, "not enough shared memory for two stages");
   static_assert(BN % CW == 0 || CW > BN, "chunking");
 };
@@ -78,12 +85,12 @@ __device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }
 
-template <int BN, bool AK, bool BKM, int EPI, typename TOUT>
+template <int BN, bool AK, bool BKM, int EPI, typename TOUT, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                    const __grid_constant__ CUtensorMap tmR, const KParams p) {
-  using C = Cfg<BN, AK, BKM, EPI, TOUT>;
+  using C = Cfg<BN, AK, BKM, EPI, TOUT, PAIR>;
   // Tiles need a 1024-byte aligned base; using the array itself (not an
   // address rounded through an integer) keeps the pointers below in the
   // shared state space, so staging accesses compile to shared, not generic,
@@ -108,6 +115,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int units = p.tiles * p.ksplit;
+  // PAIR: the two CTAs of a cluster walk the same units; rank picks the rows
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int u_first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int u_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  constexpr int TM = PAIR ? 2 * BM : BM;               // rows per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -116,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 8);
+      mbar_init(&acc_empty[a], PAIR ? 16 : 8);     // epilogue warps (of both CTAs)
     }
     mbar_init(&res_bar[0], 1);
     mbar_init(&res_bar[1], 1);
@@ -128,9 +141,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 2 * BN);
+  if (warp == 1) {
+    if (PAIR) tmem_alloc_pair(tmem_slot, 2 * BN);
+    else tmem_alloc(tmem_slot, 2 * BN);
+  }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();                    // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -141,15 +158,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued = 0;        // bit s: stage s holds a load that may be unconsumed
       uint32_t issued_par = 0;    // bit s: phase parity of that load
-      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+      for (int u = u_first; u < units && !*abort_flag; u += u_step) {
         const int tile = u % p.tiles, ks = u / p.tiles;
-        const int m0 = (tile / p.n_tiles) * BM, n0 = (tile % p.n_tiles) * BN;
+        const int m0 = (tile / p.n_tiles) * TM + (int)rank * BM, n0 = (tile % p.n_tiles) * BN;
         const int kb0 = ks * p.kb_per_split;
         const int kb1 = min(p.total_kb, kb0 + p.kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) break;
           uint8_t* sA = stages + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::A_BYTES;
+          if (PAIR) {
+            // both CTAs' bytes land on the even CTA's barrier
+            const uint32_t cfull = cluster_addr(&full[stage], 0);
+            if (leader) mbar_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+            const int nb = n0 + (int)rank * (BN / 2);
+            if (AK) {
+              tma_load_2d_pair(sA, &tmA, cfull, kb * BK, m0);
+            } else {
+              tma_load_2d_pair(sA, &tmA, cfull, m0, kb * BK);
+              tma_load_2d_pair(sA + 8192, &tmA, cfull, m0 + 64, kb * BK);
+            }
+            if (BKM) {
+              tma_load_2d_pair(sB, &tmB, cfull, kb * BK, nb);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BN / 128; ++j)
+                tma_load_2d_pair(sB + j * 8192, &tmB, cfull, nb + 64 * j, kb * BK);
+            }
+            issued |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
+          }
           mbar_expect_tx(&full[stage], C::STAGE_BYTES);
           if (AK) {
             tma_load_2d(sA, &tmA, &full[stage], kb * BK, m0);
@@ -173,20 +216,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // drain: every load this thread issued has landed before the CTA exits
+      // (PAIR: the even CTA's barriers count both CTAs' loads)
       for (int s = 0; s < C::STAGES; ++s)
-        if (issued & (1u << s)) {
+        if (leader && (issued & (1u << s))) {
           volatile int never = 0;
           mbar_wait(&full[s], (issued_par >> s) & 1u, &never, p.status);
         }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+      for (int u = u_first; u < units && !*abort_flag; u += u_step) {
         const int ks = u / p.tiles;
         const int kb0 = ks * p.kb_per_split;
         const int kb1 = min(p.total_kb, kb0 + p.kb_per_split);
@@ -206,23 +250,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = AK ? sdesc_kmajor(a0 + k * 32) : sdesc_mnmajor(a0 + k * 2048, 8192);
             const uint64_t bd = BKM ? sdesc_kmajor(b0 + k * 32) : sdesc_mnmajor(b0 + k * 2048, 8192);
-            mma_ss(d_tmem, ad, bd, C::IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+            if (PAIR) mma_ss_pair(d_tmem, ad, bd, C::IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+            else mma_ss(d_tmem, ad, bd, C::IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
           }
-          mma_commit(&empty[stage]);
+          if (PAIR) mma_commit_pair(&empty[stage], 0x3);
+          else mma_commit(&empty[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        mma_commit(&acc_full[acc]);
+        if (PAIR) mma_commit_pair(&acc_full[acc], 0x3);
+        else mma_commit(&acc_full[acc]);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
       // drain: all MMAs issued by this thread complete before TMEM is freed
-      mma_commit(done_bar);
+      if (PAIR) mma_commit_pair(done_bar, 0x1);
+      else mma_commit(done_bar);
       volatile int never = 0;
       mbar_wait(done_bar, 0, &never, p.status);
     }
@@ -239,9 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t res_phase = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const uint32_t c_acc_empty0 = PAIR ? cluster_addr(&acc_empty[0], 0) : 0u;
+    for (int u = u_first; u < units; u += u_step) {
       const int tile = u % p.tiles;
-      const int m0 = (tile / p.n_tiles) * BM, n0 = (tile % p.n_tiles) * BN;
+      const int m0 = (tile / p.n_tiles) * TM + (int)rank * BM, n0 = (tile % p.n_tiles) * BN;
       bool fail = *abort_flag != 0;
       if (!fail) fail = !mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status);
       if (named_barrier_any(bid, 128, fail)) break;
@@ -349,7 +398,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // accumulator buffer free for the MMA warp
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_cluster(c_acc_empty0 + (uint32_t)(acc * sizeof(uint64_t)));
+        else mbar_arrive(&acc_empty[acc]);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -360,9 +412,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();                    // no CTA leaves while its pair may still use it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * BN);
+    if (PAIR) tmem_dealloc_pair(tmem_base, 2 * BN);
+    else tmem_dealloc(tmem_base, 2 * BN);
   }
 }
 
@@ -380,16 +434,16 @@ int sm_count() {
   return n;
 }
 
-template <int BN, bool AK, bool BKM, int EPI, typename TOUT>
-cudaError_t run(const GemmArgs& g, uint32_t* status, cudaStream_t s) {
-  using Cf = Cfg<BN, AK, BKM, EPI, TOUT>;
+template <int BN, bool AK, bool BKM, int EPI, typename TOUT, bool PAIR>
+cudaError_t run_cfg(const GemmArgs& g, uint32_t* status, cudaStream_t s) {
+  using Cf = Cfg<BN, AK, BKM, EPI, TOUT, PAIR>;
   CUtensorMap tA, tB, tC, tC2, tR;
   memset(&tC, 0, sizeof(tC));
   memset(&tC2, 0, sizeof(tC2));
   memset(&tR, 0, sizeof(tR));
   bool ok = AK ? encode_tmap_2d(&tA, false, g.A, g.K, g.M, g.lda, 64, BM)
                : encode_tmap_2d(&tA, false, g.A, g.M, g.K, g.lda, 64, 64);
-  ok = ok && (BKM ? encode_tmap_2d(&tB, false, g.B, g.K, g.N, g.ldb, 64, BN)
+  ok = ok && (BKM ? encode_tmap_2d(&tB, false, g.B, g.K, g.N, g.ldb, 64, PAIR ? BN / 2 : BN)
                   : encode_tmap_2d(&tB, false, g.B, g.N, g.K, g.ldb, 64, 64));
   const bool o32 = sizeof(TOUT) == 4;
   if (EPI == EPI_ATOMIC_F32) {
@@ -408,7 +462,8 @@ cudaError_t run(const GemmArgs& g, uint32_t* status, cudaStream_t s) {
   p.N = g.N;
   p.K = g.K;
   p.n_tiles = (int)((g.N + BN - 1) / BN);
-  const int m_tiles = (int)((g.M + BM - 1) / BM);
+  constexpr int TMR = PAIR ? 2 * BM : BM;
+  const int m_tiles = (int)((g.M + TMR - 1) / TMR);
   p.tiles = p.n_tiles * m_tiles;
   p.total_kb = (int)((g.K + BK - 1) / BK);
   p.ksplit = 1;
@@ -425,14 +480,43 @@ cudaError_t run(const GemmArgs& g, uint32_t* status, cudaStream_t s) {
   p.status = status;
   p.has_c = g.C != nullptr;
   const int units = p.tiles * p.ksplit;
-  int grid = sm_count();
-  if (units < grid) grid = units;
-  auto kern = gemm_tc_kernel<BN, AK, BKM, EPI, TOUT>;
+  auto kern = gemm_tc_kernel<BN, AK, BKM, EPI, TOUT, PAIR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, Cf::SMEM, s>>>(tA, tB, tC, tC2, tR, p);
+  if (PAIR) {
+    // clusters of two CTAs, one pair per two SMs
+    int pairs = sm_count() / 2;
+    if (units < pairs) pairs = units;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)(2 * pairs));
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = Cf::SMEM;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, kern, tA, tB, tC, tC2, tR, p);
+    if (e != cudaSuccess) return e;
+  } else {
+    int grid = sm_count();
+    if (units < grid) grid = units;
+    kern<<<grid, kThreads, Cf::SMEM, s>>>(tA, tB, tC, tC2, tR, p);
+  }
   count_launch();
   return cudaGetLastError();
+}
+
+// 256-wide tiles on CTA pairs once there are enough rows for them (a short-K
+// residual GEMM, bound by its epilogue, stays on single CTAs)
+template <int BN, bool AK, bool BKM, int EPI, typename TOUT>
+cudaError_t run(const GemmArgs& g, uint32_t* status, cudaStream_t s) {
+  const bool pair = BN == 256 && g.M >= 2 * BM && !(EPI == EPI_RESID && g.K < 2048);
+  if (pair) return run_cfg<BN, AK, BKM, EPI, TOUT, true>(g, status, s);
+  return run_cfg<BN, AK, BKM, EPI, TOUT, false>(g, status, s);
 }
 
 template <int BN>

@@ -291,6 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = u_first; u < units; u += u_step) {
       const int tile = u % p.tiles;
       const int m0 = (tile / p.n_tiles) * TM + (int)rank * BM, n0 = (tile % p.n_tiles) * BN;
+      if (EPI == EPI_RESID && et == 0) {
+        // this warpgroup's residual chunks of the tile into L2 before the accumulator is ready
+        for (int c0 = half * C::CW; c0 < BN && c0 < p.N - n0; c0 += 2 * C::CW) tma_prefetch_2d(&tmR, n0 + c0, m0);
+      }
       bool fail = *abort_flag != 0;
       if (!fail) fail = !mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.status);
       if (named_barrier_any(bid, 128, fail)) break;

@@ -204,8 +204,9 @@ def test_proj_out_parity(dtype):
 # ----------------------------------------------------------------------------
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_proj_out_bwd_parity(dtype):
-    d = 128
+@pytest.mark.parametrize("d", [128, 512])
+def test_proj_out_bwd_parity(dtype, d):
+    # d = 512: dZ and dW2 on CTA pairs (M >= 256, 256-wide tiles), ragged M
     w = W.custom([150, 0, 81, 300], d=d, H=2, dtype=dtype, with_bias=True, backward=True)
     rng = np.random.default_rng(3)
     z = rng.normal(0, 1, size=(w.T, d)).astype(np.float32)
@@ -293,8 +294,9 @@ def test_attention_bwd_parity(dtype, dh, targets):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_proj_in_bwd_parity(dtype):
-    d = 128
+@pytest.mark.parametrize("d", [128, 512])
+def test_proj_in_bwd_parity(dtype, d):
+    # d = 512: dX (residual, K = 4d) and dW1 (split-K) on CTA pairs, ragged M
     w = W.custom([150, 0, 81, 300], d=d, H=2, dtype=dtype, with_bias=True, backward=True)
     rng = np.random.default_rng(5)
     dpre = rng.normal(0, 1, size=(w.T, 4 * d)).astype(np.float32)

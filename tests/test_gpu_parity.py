@@ -207,7 +207,8 @@ def test_proj_out_parity(dtype):
 @pytest.mark.parametrize("d", [128, 512])
 def test_proj_out_bwd_parity(dtype, d):
     # d = 512: dZ and dW2 on CTA pairs (M >= 256, 256-wide tiles), ragged M
-    w = W.custom([150, 0, 81, 300], d=d, H=2, dtype=dtype, with_bias=True, backward=True)
+    w = W.custom([150, 0, 81, 300], d=d, H=d // 128 if d > 256 else 2, dtype=dtype, with_bias=True,
+                 backward=True)
     rng = np.random.default_rng(3)
     z = rng.normal(0, 1, size=(w.T, d)).astype(np.float32)
     if dtype == "bf16":
@@ -297,7 +298,8 @@ def test_attention_bwd_parity(dtype, dh, targets):
 @pytest.mark.parametrize("d", [128, 512])
 def test_proj_in_bwd_parity(dtype, d):
     # d = 512: dX (residual, K = 4d) and dW1 (split-K) on CTA pairs, ragged M
-    w = W.custom([150, 0, 81, 300], d=d, H=2, dtype=dtype, with_bias=True, backward=True)
+    w = W.custom([150, 0, 81, 300], d=d, H=d // 128 if d > 256 else 2, dtype=dtype, with_bias=True,
+                 backward=True)
     rng = np.random.default_rng(5)
     dpre = rng.normal(0, 1, size=(w.T, 4 * d)).astype(np.float32)
     if dtype == "bf16":

@@ -841,18 +841,29 @@ __global__ void __launch_bounds__(kB3Threads, 1)
         }
         kv_iss = true;
         kv_par = items_done & 1;
-        // the next item's K and V wait for this item's last MMA: have them in L2
-        const int itn = it + gridDim.x;
-        if (itn < total) {
-          const BItem nx = P.w.items[itn];
-          const int32_t kr = (int32_t)(a.q_offsets[nx.b] + nx.kt * kT);
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            tma_prefetch_2d(&tmK, nx.h * DH + 64 * x, kr);
-            tma_prefetch_2d(&tmV, nx.h * DH + 64 * x, kr);
+      }
+      // the next item's K and V (they load only after this item's last MMA)
+      // and its first Q/dO blocks, into L2 a few blocks before this item ends
+      const int itn = it + gridDim.x;
+      auto prefetch_next = [&]() {
+        if (itn >= total) return;
+        const BItem nx = P.w.items[itn];
+        int64_t ns0;
+        int nn, nhlen;
+        bgeom(a, nx.b, ns0, nn, nhlen);
+        const int nk0 = nx.kt * kT;
+        if (lane < 4) {
+          const CUtensorMap* tm = (lane & 2) ? &tmV : &tmK;
+          tma_prefetch_2d(tm, nx.h * DH + 64 * (lane & 1), (int32_t)(ns0 + nk0));
+        } else if (lane < 4 + 4 * kPrefetch) {
+          const int mp = (lane - 4) >> 2;            // query block of the next item
+          const int qp = nk0 + mp * kQB;
+          if (qp < nn) {
+            const CUtensorMap* tm = (lane & 2) ? &tmdO : &tmQ;
+            tma_prefetch_2d(tm, nx.h * DH + 64 * (lane & 1), (int32_t)(ns0 + qp));
           }
         }
-      }
+      };
       ++items_done;
       // L2 prefetch keeps the Q, dO and time rows kPrefetch blocks ahead of
       // the loads, so that a freed stage refills at L2 rather than HBM latency
@@ -868,7 +879,9 @@ __global__ void __launch_bounds__(kB3Threads, 1)
         }
       };
       for (int mp = 1; mp < kPrefetch; ++mp) prefetch(mp);
+      if (nqb <= kPrefetch) prefetch_next();
       for (int m = 0; m < nqb; ++m, ++g) {
+        if (m == nqb - kPrefetch) prefetch_next();
         const int st = (int)(g % kQStages);
         const uint32_t par = (g / kQStages) & 1;
         const int q0 = k0 + m * kQB;

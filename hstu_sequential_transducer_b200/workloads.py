@@ -22,6 +22,9 @@ Workloads (sizes and distributions):
                    N=5120; candidates share one request time per user.
 * ``training``     bf16, 8 layers fwd+bwd; B=64, n ~ U{1024..8192}; d=1024,
                    H=8, dh=128; dY ~ N(0, 1); N=8192.
+
+``sl_draws`` gives the Stochastic Length sampler its random inputs (uint32
+keep-whole draws per sequence, uint32 ranking keys per row), uniform.
 """
 from __future__ import annotations
 
@@ -305,3 +308,14 @@ def subset(w: Workload, seqs) -> Workload:
                     backward=w.backward, microbatch=w.microbatch,
                     num_pos_buckets=w.num_pos_buckets, num_time_buckets=w.num_time_buckets,
                     ln_eps=w.ln_eps, max_seq_len=w.max_seq_len, meta=dict(w.meta))
+
+
+def sl_draws(seed: int, B: int, T: int, key_range: Optional[int] = None):
+    """Random inputs of the Stochastic Length sampler: one uint32 keep-whole
+    draw per sequence and one uint32 ranking key per input row.  A small
+    ``key_range`` forces tied keys."""
+    rng = np.random.default_rng(seed)
+    keep = rng.integers(0, 1 << 32, size=B, dtype=np.uint64).astype(np.uint32)
+    hi = (1 << 32) if key_range is None else int(key_range)
+    keys = rng.integers(0, hi, size=T, dtype=np.uint64).astype(np.uint32)
+    return keep, keys

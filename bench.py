@@ -14,6 +14,11 @@ over NCCL.  Rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on this host's cores (rank 0 only).
+
+--sampler measures the Stochastic Length sampler instead (selection plus the
+gathers of the fp32 rows and timestamps of the training batch, alpha 1.6 by
+default) and prints its own line; with --impl reference it times the oracle
+sampler on the same batch.
 """
 from __future__ import annotations
 
@@ -160,7 +165,8 @@ class ClockSampler:
 
 
 # kernel class -> the source file its traffic figure was captured from
-_KERNEL_SOURCES = {"attn_fwd": "attn_tc.cu", "attn_bwd": "attn_bwd_tc.cu"}
+_KERNEL_SOURCES = {"attn_fwd": "attn_tc.cu", "attn_bwd": "attn_bwd_tc.cu",
+                   "sl_gather": "stoch_len.cu"}
 
 
 def profiled_traffic(kernel: str, workload: str):
@@ -461,6 +467,194 @@ def e2e_training(args, ts, dw, world, dist):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
 
 
+# ----------------------------------------------------------------------------
+# Stochastic Length sampler (--sampler): its own measurement line
+# ----------------------------------------------------------------------------
+
+SAMPLER_METRIC = ("Stochastic Length sampler input tokens/s (training batch: 64 sequences "
+                  "U[1024, 8192], d=1024 fp32 rows, max_len 8192)")
+
+
+def sampler_inputs(rank: int):
+    """The training batch's lengths and timestamps (same draws as the training
+    workload), fp32 rows of width 1024 (the residual stream entering layer 1)
+    and the sampler's random inputs."""
+    seed = rank_data_seed(rank)
+    rng = np.random.default_rng(seed)
+    lengths = rng.integers(1024, 8193, size=64)
+    ts = W.draw_timestamps(rng, lengths)
+    offs = W.offsets_from_lengths(lengths)
+    T = int(offs[-1])
+    x = np.random.default_rng(seed + 1).standard_normal((T, 1024), dtype=np.float32)
+    keep, keys = W.sl_draws(seed + 2, len(lengths), T)
+    return offs, ts, x, keep, keys
+
+
+def sampler_oracle(offs, ts, x, keep, keys, L):
+    """One pass of the oracle sampler (selection, then gathers of the rows
+    and timestamps) over the whole batch; returns seconds."""
+    from oracle import stochastic_length as SL
+    t0 = time.perf_counter()
+    new_offs, gi = SL.sample(offs, None, L, keep, keys)
+    SL.gather(x, gi)
+    SL.gather(ts, gi)
+    return time.perf_counter() - t0
+
+
+def run_sampler(args):
+    import torch
+    import torch.distributed as dist
+
+    from hstu_sequential_transducer_b200 import build
+    from hstu_sequential_transducer_b200 import hstu as H
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    offs, ts, x, keep, keys = sampler_inputs(rank)
+    B, T = len(offs) - 1, int(offs[-1])
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from oracle import stochastic_length as SL
+        L = SL.subsequence_length(8192, args.alpha)
+        for _ in range(args.warmup):
+            sampler_oracle(offs, ts, x, keep, keys, L)
+        times = [sampler_oracle(offs, ts, x, keep, keys, L) for _ in range(args.steps)]
+        sec = float(np.median(times))
+        value = T / sec
+        desc = f"whole batch ({B} sequences, {T} tokens), alpha {args.alpha}"
+        print(json.dumps({
+            "metric": SAMPLER_METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1000, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+            "config": {"workload": f"stochastic_length: {desc}", "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    H.lib()
+    dev = torch.device("cuda", local)
+    L = H.sl_subsequence_length(8192, args.alpha)
+    hoffs = torch.from_numpy(offs).pin_memory()
+    hts = torch.from_numpy(ts).pin_memory()
+    hx = torch.from_numpy(x).pin_memory()
+    hkeep = torch.from_numpy(keep.view(np.int32)).pin_memory()
+    hkeys = torch.from_numpy(keys.view(np.int32)).pin_memory()
+    d_offs, d_ts, d_x = hoffs.to(dev), hts.to(dev), hx.to(dev)
+    d_keep, d_keys = hkeep.to(dev), hkeys.to(dev)
+    new_offs = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    gidx = torch.empty(T, dtype=torch.int64, device=dev)
+    x_out, ts_out = torch.empty_like(d_x), torch.empty_like(d_ts)
+    hnew = torch.empty(B + 1, dtype=torch.int64).pin_memory()
+    gather_events = []
+
+    def step(timed=False):
+        H.stochastic_length(d_offs, None, L, d_keep, d_keys, new_offs, gidx)
+        if timed:
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record()
+        H.gather_rows(d_x, gidx, new_offs[B:], x_out)
+        if timed:
+            g1.record()
+            gather_events.append((g0, g1))
+        H.gather_rows(d_ts, gidx, new_offs[B:], ts_out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t_new = int(new_offs[B].item())
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = H.launch_count()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step(timed=True)
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = H.launch_count() - launches0
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        ms = max_over_ranks(ms, dist, dev)
+    g_ms = float(np.mean([a.elapsed_time(b) for a, b in gather_events]))
+    peaks, peak_src = read_peaks()
+    # the row gather: read T' rows of 4 KiB and their indices, write T' rows
+    work = t_new * (2 * 1024 * 4 + 8)
+    ach = work / (g_ms / 1000.0) / 1e9
+    roof = {"kernel": "sl_gather", "bound": "hbm", "achieved": ach, "peak": peaks.get("hbm_gbs"),
+            "unit": "GB/s", "frac": ach / peaks.get("hbm_gbs"),
+            "traffic": profiled_traffic("sl_gather", "training"),
+            "peak_source": f"{peak_src} (hbm_gbs)", "work_per_launch": work,
+            "avg_launch_ms": g_ms}
+
+    e2e = None
+    if not args.skip_e2e:
+        def e2e_step():
+            d_offs.copy_(hoffs, non_blocking=True)
+            d_ts.copy_(hts, non_blocking=True)
+            d_x.copy_(hx, non_blocking=True)
+            d_keep.copy_(hkeep, non_blocking=True)
+            d_keys.copy_(hkeys, non_blocking=True)
+            step()
+            hnew.copy_(new_offs, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        ems = a.elapsed_time(b) / args.steps
+        if world > 1:
+            ems = max_over_ranks(ems, dist, dev)
+        h2d = (hoffs.numel() + hts.numel()) * 8 + hx.numel() * 4 + (hkeep.numel() + hkeys.numel()) * 4
+        e2e = {"value": T * world / (ems / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(hnew.numel() * 8),
+               "ms_per_step": ems}
+
+    line = {"metric": SAMPLER_METRIC, "value": T * world / (ms / 1000.0), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+            "data": "synthetic",
+            "config": {"workload": f"stochastic_length: training batch, B={B}, T={T}, "
+                                   f"alpha {args.alpha} (L={L}), sampled T'={t_new}",
+                       "global_batch": B * world, "tokens_per_step": T * world,
+                       "l2": "inputs larger than L2 (no flush)", "parallelism": f"dp{world}"},
+            "roofline": roof, "gpu_launches": launches, "clocks": clk, "e2e": e2e}
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        sec = sampler_oracle(offs, ts, x, keep, keys, L)
+        line["cpu_baseline"] = {"value": T / sec, "unit": "tokens/s", "cores": 1,
+                                "kind": "oracle", "sample": "whole batch, one pass"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -473,7 +667,12 @@ def main(argv=None):
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="keep only the first B sequences (a small case for profiler captures)")
+    ap.add_argument("--sampler", action="store_true",
+                    help="measure the Stochastic Length sampler on the training batch instead")
+    ap.add_argument("--alpha", type=float, default=1.6)
     args = ap.parse_args(argv)
+    if args.sampler:
+        return run_sampler(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -79,6 +79,9 @@ _SIGS = {
     "hstu_fwd_cached": (I32, [_CP, _WP, P, P, I32, I64, P, P, P, I64, P, P, P, S, P]),
     "hstu_bwd": (I32, [_CP, _WP, P, P, P, P, I32, I64, P, P, P, _GP, P, S, P]),
     "hstu_validate_inputs": (I32, [P, I32, I64, P, P, I32, P, P]),
+    "hstu_sl_subsequence_length": (I64, [I64, c_double]),
+    "hstu_stochastic_length": (I32, [P, P, I32, I64, I64, P, P, P, P, P]),
+    "hstu_gather_rows": (I32, [P, I64, I64, P, P, I64, I64, P, I64, P]),
     "hstu_profiler_enable": (None, [I32]),
     "hstu_profiler_collect": (I32, [I32, POINTER(c_int64), POINTER(c_double)]),
     "hstu_profiler_reset": (None, []),
@@ -325,6 +328,53 @@ def validate_inputs(offsets, timestamps, num_targets, max_seq_len, stream=None) 
                                       max_seq_len, ptr(flags), stream_ptr(stream)),
            "hstu_validate_inputs")
     return int(flags.item())
+
+
+# ----------------------------------------------------------------------------
+# Stochastic Length sampler
+# ----------------------------------------------------------------------------
+
+def sl_subsequence_length(max_len: int, alpha: float) -> int:
+    """L = floor(N^(alpha/2)), computed by the library on the host."""
+    v = int(lib().hstu_sl_subsequence_length(int(max_len), float(alpha)))
+    if v < 0:
+        raise HSTUError(1, "hstu_sl_subsequence_length")
+    return v
+
+
+def stochastic_length(offsets, num_targets, sub_len, keep_draw, keys, new_offsets=None,
+                      gather_index=None, stream=None):
+    """Samples the jagged batch; returns (new_offsets [B+1], gather_index [T])
+    on the device.  new_offsets[B] is the sampled row count; entries of
+    gather_index past it are not written."""
+    B, T = offsets.numel() - 1, keys.numel()
+    if new_offsets is None:
+        new_offsets = torch.empty(B + 1, dtype=torch.int64, device=offsets.device)
+    if gather_index is None:
+        gather_index = torch.empty(max(T, 1), dtype=torch.int64, device=offsets.device)
+    _check(lib().hstu_stochastic_length(ptr(offsets), ptr(num_targets), B, T, int(sub_len),
+                                        ptr(keep_draw), ptr(keys), ptr(new_offsets),
+                                        ptr(gather_index), stream_ptr(stream)),
+           "hstu_stochastic_length")
+    return new_offsets, gather_index
+
+
+def gather_rows(src, gather_index, d_num_rows, out, stream=None):
+    """out[r] = src[gather_index[r]] for r < d_num_rows (a device int64
+    scalar view) and r < out.shape[0]; src and out are 1-D or 2-D tensors with
+    contiguous rows of the same width and dtype."""
+    src2 = src.reshape(src.shape[0], -1)
+    out2 = out.reshape(out.shape[0], -1)
+    if src2.dtype != out2.dtype or src2.shape[1] != out2.shape[1] or \
+            src2.stride(1) != 1 or out2.stride(1) != 1:
+        raise ValueError("gather_rows: src and out need the same dtype, width and unit inner stride")
+    es = src2.element_size()
+    _check(lib().hstu_gather_rows(ptr(src2), src2.stride(0) * es, src2.shape[0],
+                                  ptr(gather_index), ptr(d_num_rows), out2.shape[0],
+                                  src2.shape[1] * es, ptr(out2), out2.stride(0) * es,
+                                  stream_ptr(stream)),
+           "hstu_gather_rows")
+    return out
 
 
 # ----------------------------------------------------------------------------

@@ -1,9 +1,10 @@
 """Device-side drivers for stacks of HSTU layers (plumbing only).
 
 Moves a seeded workload to the GPU and runs it through the C ABI: a forward
-stack, a forward+backward training step, and M-FALCON scoring (history pass
-with K/V caching, then candidate microbatches against the cache).  Every
-layer step runs in libhstu.so.
+stack, a forward+backward training step, M-FALCON scoring (history pass
+with K/V caching, then candidate microbatches against the cache), and
+Stochastic Length sampling of a training batch.  Every layer step runs in
+libhstu.so.
 """
 from __future__ import annotations
 
@@ -165,3 +166,34 @@ def mfalcon_score(dw: DeviceWorkload, history: int, candidates: int, microbatch:
         out_rows = (np.arange(B)[:, None] * candidates + k0 + np.arange(mb)[None, :]).reshape(-1)
         y_cand[torch.from_numpy(out_rows).to(dev)] = xc
     return y_hist, y_cand
+
+
+class StochasticLength:
+    """Stochastic Length sampling of a jagged batch on the device, with
+    buffers of the input's capacity allocated once.  `run` launches the
+    sampler and the row gathers without synchronising; `batch` reads the
+    sampled row count (one 8-byte device-to-host copy) and returns a
+    DeviceWorkload of the sampled batch (weights and config shared)."""
+
+    def __init__(self, dw: DeviceWorkload, alpha: float, max_len: Optional[int] = None):
+        self.dw = dw
+        self.sub_len = H.sl_subsequence_length(int(max_len or dw.cfg.max_seq_len), alpha)
+        dev = dw.x.device
+        self.new_offsets = torch.empty(dw.B + 1, dtype=torch.int64, device=dev)
+        self.gather_index = torch.empty(max(dw.T, 1), dtype=torch.int64, device=dev)
+        self.x = torch.empty_like(dw.x)
+        self.timestamps = torch.empty_like(dw.timestamps)
+
+    def run(self, keep_draw: torch.Tensor, keys: torch.Tensor, stream=None):
+        dw = self.dw
+        H.stochastic_length(dw.offsets, dw.num_targets, self.sub_len, keep_draw, keys,
+                            self.new_offsets, self.gather_index, stream=stream)
+        count = self.new_offsets[dw.B:]
+        H.gather_rows(dw.x, self.gather_index, count, self.x, stream=stream)
+        H.gather_rows(dw.timestamps, self.gather_index, count, self.timestamps, stream=stream)
+
+    def batch(self) -> DeviceWorkload:
+        dw = self.dw
+        t = int(self.new_offsets[dw.B].item())
+        return DeviceWorkload(dw.cfg, self.x[:t], self.new_offsets, self.timestamps[:t],
+                              dw.num_targets, dw.layers, None, dw.w)

@@ -300,6 +300,51 @@ hstu_status hstu_bwd(const hstu_config* cfg, const hstu_weights* w, const void* 
                      void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Stochastic Length (training-input subsampling)                            */
+/* ------------------------------------------------------------------------ */
+/* HSTU walkthrough, "Three more scaling components / Stochastic Length":
+ * training usually replaces a long history by a shorter subsequence of it and
+ * now and then keeps it whole; alpha = 1.6 maps a length of 4,096 to 776.
+ * Readings taken: the subsequence length is L = floor(N^(alpha/2)) for the
+ * maximum sequence length N; only the history (the first n - num_targets
+ * positions) is sampled and targets are always kept, after it; a history with
+ * h <= L is kept whole, a longer one is kept whole with probability L^2/h^2
+ * and is otherwise reduced to the L positions with the smallest
+ * (key, position) pairs, in their original order. */
+
+/* L = floor(N^(alpha/2)) computed on the host; -1 for N < 0, alpha < 0,
+ * alpha > 64 or NaN. */
+int64_t hstu_sl_subsequence_length(int64_t max_len, double alpha);
+
+/* Samples a jagged batch.  Inputs (device): seq_offsets int64 [B+1];
+ * num_targets int32 [B] or NULL; keep_draw uint32 [B] (sequence b is kept
+ * whole iff keep_draw[b] < (L*L / (h*h)) * 2^32, the quotient in fp64);
+ * keys uint32 [T] (one ranking key per input row; i.i.d. uniform keys give a
+ * uniform random subset).  sub_len = L >= 0.
+ * Outputs (device): new_offsets int64 [B+1] (new_offsets[B] = T', the sampled
+ * row count, T' <= T); gather_index int64 [capacity T]: output row r is input
+ * row gather_index[r], r < T'.  Build the sampled rows (embeddings,
+ * timestamps, ...) with hstu_gather_rows; num_targets is unchanged.
+ * Requires T < 2^31; int64 arrays 8-byte and uint32/int32 arrays 4-byte
+ * aligned.  Two launches, no synchronisation. */
+hstu_status hstu_stochastic_length(const int64_t* seq_offsets, const int32_t* num_targets,
+                                   int32_t B, int64_t T, int64_t sub_len,
+                                   const uint32_t* keep_draw, const uint32_t* keys,
+                                   int64_t* new_offsets, int64_t* gather_index,
+                                   cudaStream_t stream);
+
+/* dst row r = src row gather_index[r] for r < min(*d_num_rows, max_rows)
+ * (d_num_rows is a DEVICE int64, e.g. new_offsets + B, so no host sync is
+ * needed); row_bytes bytes per row, strides in bytes.  Rows whose index is
+ * outside [0, src_rows) are skipped (left unwritten).  dst must hold
+ * max_rows rows.  Copies in the widest of 16/8/4/2/1-byte vectors that the
+ * pointers, strides and row size allow. */
+hstu_status hstu_gather_rows(const void* src, int64_t src_stride_bytes, int64_t src_rows,
+                             const int64_t* gather_index, const int64_t* d_num_rows,
+                             int64_t max_rows, int64_t row_bytes, void* dst,
+                             int64_t dst_stride_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Support                                                                    */
 /* ------------------------------------------------------------------------ */
 

@@ -92,3 +92,37 @@ def test_host_argument_errors_return_before_launch(L):
     # negative sizes
     assert L.hstu_ln_gate_fwd(ctypes.byref(c), None, None, None, None, -1, None, None, None,
                               None) == 1
+
+
+def test_sl_subsequence_length_host(L):
+    """The library's host computation of L = floor(N^(alpha/2)) matches the
+    walkthrough's printed pair (alpha = 1.6: 4,096 -> 776) and the closed forms
+    in tests/golden/stochastic_length.txt."""
+    rows = [l.split() for l in open(os.path.join(ROOT, "tests", "golden", "stochastic_length.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert rows
+    for n, a, want in rows:
+        assert L.hstu_sl_subsequence_length(int(n), float(a)) == int(want), (n, a)
+    assert L.hstu_sl_subsequence_length(0, 1.6) == 0
+    assert L.hstu_sl_subsequence_length(-1, 1.6) == -1
+    assert L.hstu_sl_subsequence_length(4096, -0.5) == -1
+    assert L.hstu_sl_subsequence_length(4096, float("nan")) == -1
+
+
+def test_sl_host_argument_errors(L):
+    off = (ctypes.c_int64 * 3)()
+    a = ctypes.addressof(off)
+    # negative sizes / sub_len
+    assert L.hstu_stochastic_length(a, None, -1, 0, 5, None, None, a, None, None) == 1
+    assert L.hstu_stochastic_length(a, None, 2, 10, -1, 0x1000, 0x1000, a, 0x1000, None) == 1
+    # missing draws or outputs
+    assert L.hstu_stochastic_length(a, None, 2, 10, 5, None, 0x1000, a, 0x1000, None) == 1
+    assert L.hstu_stochastic_length(a, None, 2, 10, 5, 0x1000, 0x1000, a, None, None) == 1
+    # misaligned int64 arrays, too many rows
+    assert L.hstu_stochastic_length(a + 4, None, 2, 10, 5, 0x1000, 0x1000, a, 0x1000, None) == 2
+    assert L.hstu_stochastic_length(a, None, 2, 1 << 31, 5, 0x1000, 0x1000, a, 0x1000, None) == 2
+    # gather: empty is a no-op, bad strides and nulls are rejected
+    assert L.hstu_gather_rows(None, 0, 0, None, None, 0, 16, None, 0, None) == 0
+    assert L.hstu_gather_rows(0x1000, 8, 4, 0x2000, 0x3000, 4, 16, 0x4000, 16, None) == 1
+    assert L.hstu_gather_rows(0x1000, 16, 4, None, 0x3000, 4, 16, 0x4000, 16, None) == 1
+    assert L.hstu_gather_rows(0x1000, 16, 4, 0x2004, 0x3000, 4, 16, 0x4000, 16, None) == 2

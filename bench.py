@@ -475,14 +475,17 @@ SAMPLER_METRIC = ("Stochastic Length sampler input tokens/s (training batch: 64 
                   "U[1024, 8192], d=1024 fp32 rows, max_len 8192)")
 
 
-def sampler_inputs(rank: int):
+def sampler_inputs(rank: int, batch=None):
     """The training batch's lengths and timestamps (same draws as the training
     workload), fp32 rows of width 1024 (the residual stream entering layer 1)
-    and the sampler's random inputs."""
+    and the sampler's random inputs; `batch` keeps the first sequences."""
     seed = rank_data_seed(rank)
     rng = np.random.default_rng(seed)
     lengths = rng.integers(1024, 8193, size=64)
     ts = W.draw_timestamps(rng, lengths)
+    if batch is not None and batch < len(lengths):
+        ts = ts[:int(lengths[:batch].sum())]
+        lengths = lengths[:batch]
     offs = W.offsets_from_lengths(lengths)
     T = int(offs[-1])
     x = np.random.default_rng(seed + 1).standard_normal((T, 1024), dtype=np.float32)
@@ -511,7 +514,7 @@ def run_sampler(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    offs, ts, x, keep, keys = sampler_inputs(rank)
+    offs, ts, x, keep, keys = sampler_inputs(rank, args.batch)
     B, T = len(offs) - 1, int(offs[-1])
     if args.impl == "reference":
         if rank != 0:

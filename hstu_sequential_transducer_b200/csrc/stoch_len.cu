@@ -17,8 +17,9 @@
 //                      smallest key (four 8-bit digit passes over the keys,
 //                      which stay in L2), then an order-preserving compaction
 //                      written straight into the gather index
-//   gather_rows_kernel lane groups copy rows in 16/8/4/2/1-byte vectors; the
-//                      row count is read on the device
+//   gather_rows_*      warps (wide rows) or lane groups (narrow rows) copy
+//                      rows in 16/8/4/2/1-byte vectors; the row count is
+//                      read on the device
 #include <math.h>
 
 #include "common.cuh"
@@ -238,6 +239,52 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
   }
 }
 
+// Wide rows (at least 32 vectors): the work is split into units of one
+// 32-vector segment of a row, dealt to warps round-robin (unit u = row * segs
+// + seg goes to warp u mod warps), so that the last round leaves at most one
+// unit per warp idle instead of one row.  Each warp keeps four units' loads
+// in flight before storing; (row, seg) advance incrementally, with no
+// division in the loop.
+template <typename V>
+__global__ void __launch_bounds__(256) gather_rows_wide_kernel(
+    const unsigned char* __restrict__ src, int64_t src_ld, int64_t src_rows,
+    const int64_t* __restrict__ index, const int64_t* __restrict__ n_rows, int64_t max_rows,
+    int64_t vecs_per_row, int64_t segs, unsigned char* __restrict__ dst, int64_t dst_ld) {
+  constexpr int kInFlight = 4;
+  int64_t rows = *n_rows;
+  if (rows > max_rows) rows = max_rows;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  int64_t row = warp0 / segs, seg = warp0 - (warp0 / segs) * segs;
+  const int64_t drow = nwarps / segs, dseg = nwarps - drow * segs;
+  while (row < rows) {
+    V v[kInFlight];
+    V* dp[kInFlight];
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      dp[k] = nullptr;
+      if (row < rows) {
+        const int64_t q = seg * 32 + lane;
+        const int64_t sr = index[row];
+        if (q < vecs_per_row && sr >= 0 && sr < src_rows) {
+          v[k] = reinterpret_cast<const V*>(src + sr * src_ld)[q];
+          dp[k] = reinterpret_cast<V*>(dst + row * dst_ld) + q;
+        }
+      }
+      seg += dseg;
+      row += drow;
+      if (seg >= segs) {
+        seg -= segs;
+        ++row;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k)
+      if (dp[k]) *dp[k] = v[k];
+  }
+}
+
 template <typename V>
 cudaError_t launch_gather(const void* src, int64_t src_ld, int64_t src_rows, const int64_t* index,
                           const int64_t* n_rows, int64_t max_rows, int64_t row_bytes, void* dst,
@@ -254,10 +301,19 @@ cudaError_t launch_gather(const void* src, int64_t src_ld, int64_t src_rows, con
   };
   const auto* sp = static_cast<const unsigned char*>(src);
   auto* dp = static_cast<unsigned char*>(dst);
-  if (vecs >= 32)
-    gather_rows_kernel<V, 32><<<grid(8), 256, 0, s>>>(sp, src_ld, src_rows, index, n_rows,
-                                                      max_rows, vecs, dp, dst_ld);
-  else if (vecs >= 8)
+  if (vecs >= 32) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gather_rows_wide_kernel<V>, 256,
+                                                      0) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    const int64_t segs = (vecs + 31) / 32;
+    const int64_t units_cap = max_rows * segs;            // warps beyond this have no work
+    int64_t g = (units_cap + 7) / 8;
+    const int64_t cap = (int64_t)sms * per_sm;
+    g = g < 1 ? 1 : (g > cap ? cap : g);
+    gather_rows_wide_kernel<V><<<(unsigned)g, 256, 0, s>>>(sp, src_ld, src_rows, index, n_rows,
+                                                            max_rows, vecs, segs, dp, dst_ld);
+  } else if (vecs >= 8)
     gather_rows_kernel<V, 8><<<grid(32), 256, 0, s>>>(sp, src_ld, src_rows, index, n_rows,
                                                       max_rows, vecs, dp, dst_ld);
   else

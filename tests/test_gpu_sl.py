@@ -105,7 +105,8 @@ def test_sl_edge_cases(case):
     check(offs, nt, L, keep, keys)
 
 
-@pytest.mark.parametrize("kind", ["bf16_d1024", "f32_d1024", "i64_ts", "f32_d50", "u8_3"])
+@pytest.mark.parametrize("kind", ["bf16_d1024", "f32_d1024", "f32_d1000", "i64_ts", "f32_d50",
+                                  "u8_3"])
 def test_sl_gather_rows(kind):
     rng = np.random.default_rng(9)
     lengths = rng.integers(200, 2500, size=20)
@@ -120,6 +121,9 @@ def test_sl_gather_rows(kind):
         xt = torch.from_numpy(x).to(DEV).to(torch.bfloat16)
     elif kind == "f32_d1024":
         x = rng.standard_normal((T, 1024)).astype(np.float32)
+        xt = torch.from_numpy(x).to(DEV)
+    elif kind == "f32_d1000":  # 250 16-byte vectors: a ragged last segment
+        x = rng.standard_normal((T, 1000)).astype(np.float32)
         xt = torch.from_numpy(x).to(DEV)
     elif kind == "i64_ts":
         x = W.draw_timestamps(rng, lengths)

@@ -362,6 +362,48 @@ def test_long_history_subset_bf16():
     check(y[n_small:n_small + pref], oracle_stack(longest), "bf16", "Y long_history prefix")
 
 
+def test_long_history_full_size_sampled():
+    """The whole long-history workload (32 sequences up to 8,192 tokens, 4
+    layers) in one launch configuration; sampled against the oracle: the two
+    shortest sequences whole and the longest on its first 384 tokens
+    (sequences are independent and the mask is causal, so a prefix's output
+    is the output of the prefix alone)."""
+    w = W.long_history()
+    dw = S.DeviceWorkload.from_workload(w)
+    y = np_(S.forward_stack(dw))
+    order = np.argsort(w.lengths)
+    for b in sorted(order[:2].tolist()):
+        s, e = int(w.seq_offsets[b]), int(w.seq_offsets[b + 1])
+        check(y[s:e], oracle_stack(W.subset(w, [b])), "bf16", f"Y long_history seq {b}")
+    b = int(order[-1])
+    longest = W.subset(w, [b])
+    pref = 384
+    longest.x, longest.timestamps = longest.x[:pref], longest.timestamps[:pref]
+    longest.seq_offsets = np.array([0, pref], np.int64)
+    s = int(w.seq_offsets[b])
+    check(y[s:s + pref], oracle_stack(longest), "bf16", "Y long_history longest prefix")
+
+
+def test_mfalcon_full_size_sampled():
+    """The whole M-FALCON workload (16 users x (4,096 history + 1,024
+    candidates), 3 layers, microbatches of 256) as the benchmark scores it;
+    user 0's history rows and 16 of its candidates (the first and last 8:
+    microbatches 0 and 3) against the oracle's cached pass, whose candidate
+    scores depend on no other candidate."""
+    w = W.mfalcon()
+    dw = S.DeviceWorkload.from_workload(w)
+    hist, cand = w.meta["history"], w.meta["candidates"]
+    y_hist, y_cand = S.mfalcon_score(dw, hist, cand, w.microbatch)
+    plist = [lp(p) for p in w.params]
+    ref_hist, cache = R.mfalcon_history(w.x[:hist], w.timestamps[:hist], plist, lcfg(w))
+    idx = np.r_[0:8, cand - 8:cand]
+    ref_cand = R.mfalcon_candidates(w.x[hist + idx], w.timestamps[hist + idx], cache, plist,
+                                    lcfg(w))
+    check(np_(y_hist[:hist]), ref_hist, "bf16", "Y history, user 0 (full size)")
+    check(np_(y_cand[torch.from_numpy(idx).cuda()]), ref_cand, "bf16",
+          "Y candidates, user 0 (full size)")
+
+
 def test_layer_fwd_bwd_parity_small():
     for dtype in ("f32", "bf16"):
         w = W.custom([70, 1, 0, 130, 33], d=128, H=2, dtype=dtype, N=120.0, num_targets=[5, 0, 0, 20, 33],

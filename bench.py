@@ -700,6 +700,142 @@ def run_sampler(args):
     return 0
 
 
+# ----------------------------------------------------------------------------
+# The attention kernels alone at length 8,192 (--attention-8k)
+# ----------------------------------------------------------------------------
+
+ATTN8K_METRIC = ("HSTU attention fwd+bwd TFLOP/s at length 8192 (16 x 8192 tokens, H=8, dh=128, "
+                 "causal, pos+time rab, bf16)")
+
+
+def attn8k_oracle(seconds: float):
+    """The oracle's attention forward and backward on 1,024-token prefixes
+    (d = 1,024, H = 8) for about `seconds`; returns (algorithmic TFLOP/s,
+    sample description)."""
+    from oracle import hstu_ref as R
+    rng = np.random.default_rng(41)
+    n, d, H = 1024, 1024, 8
+    offs = np.array([0, n], np.int64)
+    ts = W.draw_timestamps(rng, [n])
+    g = rng.standard_normal((n, 4 * d)) * 0.5
+    do = rng.standard_normal((n, d))
+    rp, rt = rng.normal(0, 0.1, (H, 32)), rng.normal(0, 0.1, (H, 32))
+    cfg = R.LayerConfig(H, 8192.0, 32, 32, 1e-5)
+    t_used, reps = 0.0, 0
+    while t_used < seconds or reps == 0:
+        t0 = time.perf_counter()
+        R.attention_forward(g, offs, ts, None, rp, rt, cfg)
+        R.attention_backward(g, do, offs, ts, None, rp, rt, cfg)
+        t_used += time.perf_counter() - t0
+        reps += 1
+    flops = 12 * d * (n * (n + 1) // 2) * reps
+    return flops / t_used / 1e12, f"{reps} x one 1,024-token sequence, fwd+bwd, d=1024, H=8"
+
+
+def run_attention8k(args):
+    import torch
+
+    from hstu_sequential_transducer_b200 import build
+    from hstu_sequential_transducer_b200 import hstu as H
+
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        v, desc = attn8k_oracle(args.cpu_budget)
+        print(json.dumps({
+            "metric": ATTN8K_METRIC, "value": v, "unit": "TFLOP/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"attention at 8192: {desc}", "parallelism": "host cores"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    build.build()
+    H.lib()
+    dev = torch.device("cuda", local)
+    B, n, d, nh = 16, 8192, 1024, 8
+    T = B * n
+    rng = np.random.default_rng(7 + rank)
+    cfg = H.make_config(d, nh, 8192.0, H.HSTU_BF16, 32, 32, 8192)
+    offs = torch.arange(B + 1, dtype=torch.int64, device=dev) * n
+    ts = torch.from_numpy(W.draw_timestamps(rng, [n] * B)).to(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11 + rank)
+    g = (torch.randn(T, 4 * d, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
+    pre = torch.randn(T, 4 * d, device=dev, generator=gen).to(torch.bfloat16)
+    dout = torch.randn(T, d, device=dev, generator=gen).to(torch.bfloat16)
+    rab_pos = torch.from_numpy(rng.normal(0, 0.1, (nh, 32)).astype(np.float32)).to(dev)
+    rab_time = torch.from_numpy(rng.normal(0, 0.1, (nh, 32)).astype(np.float32)).to(dev)
+    o = torch.empty(T, d, dtype=torch.float32, device=dev)
+    dpre = torch.zeros(T, 4 * d, dtype=torch.bfloat16, device=dev)
+    drp, drt = torch.zeros_like(rab_pos), torch.zeros_like(rab_time)
+    pairs = B * n * (n + 1) // 2
+    f_fwd, f_bwd = 4 * d * pairs, 8 * d * pairs
+    ev = []
+
+    def step(timed=False):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if timed else None
+        if timed:
+            e[0].record()
+        H.attention_fwd(cfg, rab_pos, rab_time, g, offs, ts, None, o)
+        if timed:
+            e[1].record()
+        H.attention_bwd(cfg, rab_pos, rab_time, g, pre, dout, offs, ts, None, dpre, drp, drt)
+        if timed:
+            e[2].record()
+            ev.append(e)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = H.launch_count()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step(timed=True)
+    e1.record()
+    torch.cuda.synchronize()
+    launches = H.launch_count() - launches0
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    fwd_ms = float(np.median([a.elapsed_time(b) for a, b, _ in ev]))
+    bwd_ms = float(np.median([b.elapsed_time(c) for _, b, c in ev]))
+    peaks, peak_src = read_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    fwd_tf, bwd_tf = f_fwd / fwd_ms / 1e9, f_bwd / bwd_ms / 1e9
+    line = {"metric": ATTN8K_METRIC, "value": (f_fwd + f_bwd) / ms / 1e9, "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "attention at 8192: B=16 sequences of 8,192 tokens, d=1024, "
+                                   "H=8, dh=128, causal, 32+32 rab buckets, N=8192",
+                       "tokens_per_step": T, "l2": "inputs larger than L2 (no flush)",
+                       "parallelism": "dp1"},
+            "attn_fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
+            "attn_bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
+            "roofline": {"kernel": "attn_bwd", "bound": "tensor", "achieved": bwd_tf, "peak": peak,
+                         "unit": "TFLOP/s", "frac": bwd_tf / peak, "traffic": None,
+                         "peak_source": f"{peak_src} (bf16_tflops_sustained)",
+                         "work_per_launch": f_bwd},
+            "gpu_launches": launches, "clocks": clk, "e2e": None}
+    if not args.skip_cpu:
+        v, desc = attn8k_oracle(args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -715,7 +851,11 @@ def main(argv=None):
     ap.add_argument("--sampler", action="store_true",
                     help="measure the Stochastic Length sampler on the training batch instead")
     ap.add_argument("--alpha", type=float, default=1.6)
+    ap.add_argument("--attention-8k", action="store_true",
+                    help="measure the attention kernels alone on 16 sequences of 8,192 tokens")
     args = ap.parse_args(argv)
+    if args.attention_8k:
+        return run_attention8k(args)
     if args.sampler:
         return run_sampler(args)
     if args.impl == "reference":

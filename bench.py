@@ -15,6 +15,9 @@ over NCCL.  Rank 0 prints one JSON line.
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on this host's cores (rank 0 only).
 
+--attention-8k measures the two attention kernels alone on 16 sequences of
+exactly 8,192 tokens (H=8, dh=128) and prints their TFLOP/s on its own line.
+
 --sampler measures the Stochastic Length sampler instead (selection plus the
 gathers of the fp32 rows and timestamps of the training batch, alpha 1.6 by
 default) and prints its own line; with --impl reference it times the oracle

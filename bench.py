@@ -758,6 +758,8 @@ def run_attention8k(args):
                     "d2h_bytes_per_step": 0}}), flush=True)
         return 0
 
+    if rank != 0:          # a single-GPU measurement: under torchrun only rank 0 runs it
+        return 0
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     build.build()

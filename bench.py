@@ -765,7 +765,7 @@ def run_attention8k(args):
     build.build()
     H.lib()
     dev = torch.device("cuda", local)
-    B, n, d, nh = 16, 8192, 1024, 8
+    B, n, d, nh = (args.batch or 16), 8192, 1024, 8
     T = B * n
     rng = np.random.default_rng(7 + rank)
     cfg = H.make_config(d, nh, 8192.0, H.HSTU_BF16, 32, 32, 8192)
@@ -822,7 +822,7 @@ def run_attention8k(args):
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "attention at 8192: B=16 sequences of 8,192 tokens, d=1024, "
+            "config": {"workload": f"attention at 8192: B={B} sequences of 8,192 tokens, d=1024, "
                                    "H=8, dh=128, causal, 32+32 rab buckets, N=8192",
                        "tokens_per_step": T, "l2": "inputs larger than L2 (no flush)",
                        "parallelism": "dp1"},

@@ -42,6 +42,7 @@ sys.path.insert(0, ROOT)
 from hstu_sequential_transducer_b200 import workloads as W  # noqa: E402
 
 METRIC = "HSTU layer fwd+bwd tokens/s and TFLOP/s at max_len 8192; % of B200 BF16 peak"
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def pairs_allowed(lengths, num_targets=None):
@@ -381,6 +382,26 @@ def run_ours(args):
         # read dZ, O (fp32), U, Pre_U, statistics; write dO and dPre_U
         "ln_bwd": ("hbm", w.T * (14 * d + 8)),
     }
+    # contractions that run on the FP32 pipes (fp32 layers; attention at
+    # dh = 32) are held against the FP32 FMA peak: 148 SMs x 128 lanes x
+    # 2 flops x 1.965 GHz = 74.4 TFLOP/s
+    dh = d // w.num_heads
+    if w.dtype == "f32" or dh == 32:
+        for k in ("attn_fwd", "attn_bwd"):
+            per_launch[k] = ("alu", per_launch[k][1])
+    if w.dtype == "f32":
+        for k in ("proj_in", "proj_out", "proj_in_bwd", "proj_out_bwd"):
+            per_launch[k] = ("alu", per_launch[k][1])
+    if args.workload == "mfalcon" and args.batch is None:
+        # the history pass runs attn_fwd (causal over each user's history);
+        # each candidate microbatch runs attn_cached (history + self per
+        # candidate); the projections see history and microbatch rows
+        hist, cand, mb = w.meta["history"], w.meta["candidates"], w.microbatch
+        per_launch["attn_fwd"] = ("tensor", 4 * d * w.B * hist * (hist + 1) // 2)
+        per_launch["attn_cached"] = ("tensor", 4 * d * w.B * mb * (hist + 1))
+        per_launch.pop("proj_in")
+        per_launch.pop("proj_out")
+        per_launch.pop("ln_fwd")
     roof = None
     if kern:
         top = max((k for k in kern if k in per_launch), key=lambda k: kern[k]["total_ms"],
@@ -391,15 +412,18 @@ def run_ours(args):
             if bound == "tensor":
                 ach = work / avg_s / 1e12
                 peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-                unit = "TFLOP/s"
+                unit, src = "TFLOP/s", f"{peak_src} (bf16_tflops_sustained)"
+            elif bound == "alu":
+                ach = work / avg_s / 1e12
+                peak = FP32_FMA_TFLOPS
+                unit, src = "TFLOP/s", "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"
             else:
                 ach = work / avg_s / 1e9
                 peak = peaks.get("hbm_gbs")
-                unit = "GB/s"
+                unit, src = "GB/s", f"{peak_src} (hbm_gbs)"
             roof = {"kernel": top, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
                     "frac": ach / peak, "traffic": profiled_traffic(top, w.name),
-                    "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if bound == 'tensor' else 'hbm_gbs'})",
-                    "work_per_launch": work}
+                    "peak_source": src, "work_per_launch": work}
 
     # end to end through the public API with host buffers
     e2e = None

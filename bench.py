@@ -104,15 +104,19 @@ def max_over_ranks(ms: float, dist, device) -> float:
     return float(t.item())
 
 
-def make_workload(name, rank, batch=None):
-    """The named workload; `batch` keeps only its first sequences (a small
-    case of the same shapes, e.g. for profiler captures)."""
+def make_workload(name, rank, batch=None, layers=None):
+    """The named workload; `batch` keeps only its first sequences and
+    `layers` its first layers (a small case of the same shapes, e.g. for
+    profiler captures)."""
     if name == "training":
         w = W.training(data_seed=rank_data_seed(rank))
     else:
         w = W.WORKLOADS[name]()
     if batch is not None and batch < w.B:
         w = W.subset(w, list(range(batch)))
+    if layers is not None and layers < w.num_layers:
+        w.params = w.params[:layers]
+        w.num_layers = layers
     return w
 
 
@@ -255,7 +259,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = make_workload(args.workload, 0, args.batch)
+    w = make_workload(args.workload, 0, args.batch, args.layers)
     for _ in range(args.warmup):
         oracle_sample(w, 0.0)
     vals, times = [], []
@@ -304,7 +308,7 @@ def run_ours(args):
         dist.barrier()
     H.lib()
 
-    w = make_workload(args.workload, rank, args.batch)
+    w = make_workload(args.workload, rank, args.batch, args.layers)
     dw = S.DeviceWorkload.from_workload(w)
     backward = w.backward
     flops, pairs = workload_flops(w, backward)
@@ -877,6 +881,8 @@ def main(argv=None):
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="keep only the first B sequences (a small case for profiler captures)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="keep only the first L layers (a small case for profiler captures)")
     ap.add_argument("--sampler", action="store_true",
                     help="measure the Stochastic Length sampler on the training batch instead")
     ap.add_argument("--alpha", type=float, default=1.6)

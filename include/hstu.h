@@ -337,8 +337,8 @@ hstu_status hstu_stochastic_length(const int64_t* seq_offsets, const int32_t* nu
  * (d_num_rows is a DEVICE int64, e.g. new_offsets + B, so no host sync is
  * needed); row_bytes bytes per row, strides in bytes.  Rows whose index is
  * outside [0, src_rows) are skipped (left unwritten).  dst must hold
- * max_rows rows.  Copies in the widest of 16/8/4/2/1-byte vectors that the
- * pointers, strides and row size allow. */
+ * max_rows rows and must not overlap src.  Copies in the widest of
+ * 16/8/4/2/1-byte vectors that the pointers, strides and row size allow. */
 hstu_status hstu_gather_rows(const void* src, int64_t src_stride_bytes, int64_t src_rows,
                              const int64_t* gather_index, const int64_t* d_num_rows,
                              int64_t max_rows, int64_t row_bytes, void* dst,

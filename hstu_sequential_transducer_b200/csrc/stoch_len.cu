@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(1024) sl_offsets_kernel(const int64_t* __restr
     int64_t len = 0;
     if (b < B) {
       const int64_t n = offs[b + 1] - offs[b];
-      const int64_t m = nt ? (int64_t)nt[b] : 0;
+      const int64_t m = nt ? min(max((int64_t)nt[b], (int64_t)0), n) : 0;  // in [0, n]
       len = sl_keep_whole(n - m, L, keep[b]) ? n : L + m;
     }
     int64_t v = len;
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kSelThreads) sl_select_kernel(
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
   const int64_t s = offs[b], n = offs[b + 1] - s;
-  const int64_t m = nt ? (int64_t)nt[b] : 0;
+  const int64_t m = nt ? min(max((int64_t)nt[b], (int64_t)0), n) : 0;  // in [0, n]
   const int64_t h = n - m;
   const int64_t o = new_offs[b];
   const int64_t out_n = new_offs[b + 1] - o;

@@ -348,6 +348,13 @@ def stochastic_length(offsets, num_targets, sub_len, keep_draw, keys, new_offset
     on the device.  new_offsets[B] is the sampled row count; entries of
     gather_index past it are not written."""
     B, T = offsets.numel() - 1, keys.numel()
+    for name, t, sizes in (("offsets", offsets, (8,)), ("keep_draw", keep_draw, (4,)),
+                           ("keys", keys, (4,)), ("num_targets", num_targets, (4,))):
+        if t is not None and (t.element_size() not in sizes or not t.is_contiguous()):
+            raise ValueError(f"stochastic_length: {name} must be contiguous with "
+                             f"{sizes[0]}-byte elements")
+    if keep_draw.numel() != B:
+        raise ValueError("stochastic_length: keep_draw needs one entry per sequence")
     if new_offsets is None:
         new_offsets = torch.empty(B + 1, dtype=torch.int64, device=offsets.device)
     if gather_index is None:

@@ -126,3 +126,16 @@ def test_sl_host_argument_errors(L):
     assert L.hstu_gather_rows(0x1000, 8, 4, 0x2000, 0x3000, 4, 16, 0x4000, 16, None) == 1
     assert L.hstu_gather_rows(0x1000, 16, 4, None, 0x3000, 4, 16, 0x4000, 16, None) == 1
     assert L.hstu_gather_rows(0x1000, 16, 4, 0x2004, 0x3000, 4, 16, 0x4000, 16, None) == 2
+
+
+def test_sl_binding_rejects_wrong_dtypes(L):
+    import torch
+    offs = torch.zeros(3, dtype=torch.int64)
+    keep = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        H.stochastic_length(offs, None, 5, keep, torch.zeros(4, dtype=torch.int64))
+    with pytest.raises(ValueError):
+        H.stochastic_length(offs.to(torch.int32), None, 5, keep, torch.zeros(4, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        H.stochastic_length(offs, None, 5, torch.zeros(3, dtype=torch.int32),
+                            torch.zeros(4, dtype=torch.int32))

@@ -182,3 +182,33 @@ def test_sl_then_layer_forward():
     got = y.double().cpu().numpy()
     rms = np.sqrt(np.mean(want ** 2))
     assert np.max(np.abs(got - want)) <= 1e-4 * rms
+
+
+def test_sl_then_train_step():
+    """A training step (fwd + bwd, 2 layers) on a sampled batch against the
+    oracle's forward and backward on the oracle-sampled batch."""
+    from oracle import hstu_ref as R
+    from hstu_sequential_transducer_b200 import stack as S
+    rng = np.random.default_rng(31)
+    lengths = rng.integers(60, 300, size=6)
+    w = W.custom(lengths, d=64, H=2, N=300.0, dtype="f32", layers=2, seed=37, backward=True)
+    dw = S.DeviceWorkload.from_workload(w)
+    sl = S.StochasticLength(dw, alpha=1.6, max_len=300)
+    keep, keys = W.sl_draws(41, w.B, w.T)
+    sl.run(torch.from_numpy(keep.view(np.int32)).to(DEV),
+           torch.from_numpy(keys.view(np.int32)).to(DEV))
+    batch = sl.batch()
+    new_offs, gi = SL.sample(w.seq_offsets, None, sl.sub_len, keep, keys)
+    dy = w.dy[gi]
+    step = S.TrainStep(batch)
+    step.zero_grads()
+    dx = step.run(torch.from_numpy(dy).to(DEV))
+    torch.cuda.synchronize()
+    plist = [R.LayerParams(p.W1, p.W2, p.rab_pos, p.rab_time, p.b1, p.b2, p.gamma, p.beta)
+             for p in w.params]
+    cfg = R.LayerConfig(w.num_heads, w.norm_N, w.num_pos_buckets, w.num_time_buckets, w.ln_eps)
+    y, rdx, rgr = R.stack_forward_backward(SL.gather(w.x, gi), new_offs, SL.gather(w.timestamps, gi),
+                                           None, plist, cfg, dy)
+    for got, ref in ((step.y, y), (dx, rdx), (step.grads[0].dW1, rgr[0].dW1)):
+        got = got.double().cpu().numpy()
+        assert np.max(np.abs(got - ref)) <= 1e-4 * np.sqrt(np.mean(ref ** 2)) * 3

@@ -214,3 +214,23 @@ def test_sl_then_train_step():
     for got, ref in ((step.y, y), (dx, rdx), (step.grads[0].dW1, rgr[0].dW1)):
         got = got.double().cpu().numpy()
         assert np.max(np.abs(got - ref)) <= 1e-4 * np.sqrt(np.mean(ref ** 2)) * 3
+
+
+def test_gather_rows_skips_out_of_range_indices():
+    """Indices outside [0, src_rows) leave their output rows unwritten (the
+    documented behaviour of hstu_gather_rows); the row count comes from the
+    device and caps at max_rows."""
+    src = torch.arange(40 * 12, dtype=torch.float32, device=DEV).reshape(40, 12)
+    idx = torch.tensor([3, -1, 39, 40, 7, 1 << 40, 0, 5], dtype=torch.int64, device=DEV)
+    count = torch.tensor([7], dtype=torch.int64, device=DEV)      # the last index is not used
+    out = torch.full((8, 12), -5.0, dtype=torch.float32, device=DEV)
+    H.gather_rows(src, idx, count, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    s = src.cpu().numpy()
+    for r, i in enumerate([3, -1, 39, 40, 7, 1 << 40, 0]):
+        if 0 <= i < 40:
+            np.testing.assert_array_equal(got[r], s[i])
+        else:
+            assert (got[r] == -5.0).all()
+    assert (got[7] == -5.0).all()

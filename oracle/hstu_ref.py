@@ -28,7 +28,7 @@ Recommendations", arXiv 2402.17152):
   "Serving it: M-FALCON" (history work computed once and cached, candidates
   scored in microbatches against it).
 
-Readings where the pages are silent (each also listed in the design notes):
+Readings where the pages are silent:
 
 * The pooled value is scaled by 1/N with N a per-configuration constant (not
   the sequence length); Q K^T carries no 1/sqrt(dh) factor.
@@ -77,11 +77,15 @@ def silu_grad(x):
 def bit_length(v):
     """Exact integer bit length of non-negative int64 values (0 -> 0,
     1 -> 1, 2..3 -> 2, 4..7 -> 3, ...), without floating-point logarithms."""
+    # binary search over the exponent: at each step, if v has a bit at or
+    # above 2^k, count k bits and shift them out (integer arithmetic only)
     v = np.asarray(v, dtype=np.int64)
     out = np.zeros(v.shape, dtype=np.int64)
-    for k in range(63):
-        out += (v >= (np.int64(1) << np.int64(k))).astype(np.int64)
-    return out
+    for k in (32, 16, 8, 4, 2, 1):
+        big = v >= (np.int64(1) << np.int64(k))
+        out += big * np.int64(k)
+        v = np.where(big, v >> np.int64(k), v)
+    return out + (v > 0)
 
 
 def time_bucket(dt, num_buckets):
@@ -491,13 +495,15 @@ def attention_forward(g, seq_offsets, timestamps, num_targets, rab_pos, rab_time
         n = e - s
         m = 0 if num_targets is None else int(num_targets[b])
         mask = allowed_mask(n, m)
+        bp, bt = bucket_ids(n, m, ts[s:e], cfg.num_pos_buckets, cfg.num_time_buckets)
         _, V, Q, K = _split(g[s:e], d)
         for hh in range(H):
             cs = slice(hh * dh, (hh + 1) * dh)
-            bias = rab_bias(n, m, ts[s:e],
-                            None if rab_pos is None else rab_pos[hh],
-                            None if rab_time is None else rab_time[hh],
-                            cfg.num_pos_buckets, cfg.num_time_buckets)
+            bias = np.zeros((n, n))
+            if rab_pos is not None:
+                bias = bias + np.asarray(rab_pos[hh], F64)[bp]
+            if rab_time is not None:
+                bias = bias + np.asarray(rab_time[hh], F64)[bt]
             S = Q[:, cs] @ K[:, cs].T + bias
             o[s:e, cs] = (np.where(mask, silu(S), 0.0) / cfg.norm_N) @ V[:, cs]
     return o

@@ -16,7 +16,7 @@ of the time because attention cost grows with the square of the length (the
 walkthrough's section "Why user-level generative training saves a factor"
 writes attention as O(N^2 d) for a maximum length N).
 
-Readings where the pages are silent (each also listed in the design notes):
+Readings where the pages are silent:
 
 * Subsequence length L = floor(N^(alpha/2)) with N the maximum sequence
   length of the configuration.  This is the one reading that reproduces the

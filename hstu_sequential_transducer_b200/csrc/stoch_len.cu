@@ -39,9 +39,19 @@ __device__ __forceinline__ bool sl_keep_whole(int64_t h, int64_t L, uint32_t dra
   return (double)draw < p * 4294967296.0;
 }
 
+// Rows [s, s + n) of sequence b with both ends clamped into [0, T], so that
+// malformed offsets (decreasing, negative or past T) never move a read or a
+// write outside the T rows of keys and of the gather index.
+__device__ __forceinline__ void sl_rows(const int64_t* __restrict__ offs, int64_t b, int64_t T,
+                                        int64_t& s, int64_t& n) {
+  s = min(max(offs[b], (int64_t)0), T);
+  const int64_t e = min(max(offs[b + 1], s), T);
+  n = e - s;
+}
+
 __global__ void __launch_bounds__(1024) sl_offsets_kernel(const int64_t* __restrict__ offs,
                                                           const int32_t* __restrict__ nt, int B,
-                                                          int64_t L,
+                                                          int64_t T, int64_t L,
                                                           const uint32_t* __restrict__ keep,
                                                           int64_t* __restrict__ new_offs) {
   __shared__ int64_t warp_tot[32];
@@ -56,7 +66,8 @@ __global__ void __launch_bounds__(1024) sl_offsets_kernel(const int64_t* __restr
     const int64_t b = base + (int64_t)threadIdx.x;
     int64_t len = 0;
     if (b < B) {
-      const int64_t n = offs[b + 1] - offs[b];
+      int64_t s0, n;
+      sl_rows(offs, b, T, s0, n);
       const int64_t m = nt ? min(max((int64_t)nt[b], (int64_t)0), n) : 0;  // in [0, n]
       len = sl_keep_whole(n - m, L, keep[b]) ? n : L + m;
     }
@@ -116,7 +127,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t* red, u
 
 __global__ void __launch_bounds__(kSelThreads) sl_select_kernel(
     const int64_t* __restrict__ offs, const int32_t* __restrict__ nt,
-    const uint32_t* __restrict__ keys, const int64_t* __restrict__ new_offs, int64_t L,
+    const uint32_t* __restrict__ keys, const int64_t* __restrict__ new_offs, int64_t T, int64_t L,
     int64_t* __restrict__ gidx) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t red[kSelWarps];
@@ -124,18 +135,24 @@ __global__ void __launch_bounds__(kSelThreads) sl_select_kernel(
   __shared__ int64_t s_below;
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
-  const int64_t s = offs[b], n = offs[b + 1] - s;
+  int64_t s, n;
+  sl_rows(offs, b, T, s, n);
   const int64_t m = nt ? min(max((int64_t)nt[b], (int64_t)0), n) : 0;  // in [0, n]
   const int64_t h = n - m;
   const int64_t o = new_offs[b];
   const int64_t out_n = new_offs[b + 1] - o;
+  // the gather index holds T entries; with well-formed offsets every write
+  // lands inside it, and the check keeps malformed ones from writing past it
+  auto put = [&](int64_t at, int64_t row) {
+    if (at >= 0 && at < T) gidx[at] = row;
+  };
 
   if (out_n == n) {  // kept whole (always so when h <= L)
-    for (int64_t j = tid; j < n; j += kSelThreads) gidx[o + j] = s + j;
+    for (int64_t j = tid; j < n; j += kSelThreads) put(o + j, s + j);
     return;
   }
   // Sampled: out_n == L + m with L < h.  Targets go after the L history rows.
-  for (int64_t j = tid; j < m; j += kSelThreads) gidx[o + L + j] = s + h + j;
+  for (int64_t j = tid; j < m; j += kSelThreads) put(o + L + j, s + h + j);
   if (L == 0) return;
 
   const uint32_t* kb = keys + s;
@@ -209,7 +226,7 @@ __global__ void __launch_bounds__(kSelThreads) sl_select_kernel(
     const bool sel = lt || (eq && eq_rank < take_eq);
     if (sel) {
       const int64_t pos = run_lt + (before & 0xffffu) + (eq_rank < take_eq ? eq_rank : take_eq);
-      gidx[o + pos] = s + j;
+      put(o + pos, s + j);
     }
     run_lt += total & 0xffffu;
     run_eq += total >> 16;
@@ -360,13 +377,13 @@ hstu_status hstu_stochastic_length(const int64_t* seq_offsets, const int32_t* nu
       (gather_index && !addr_multiple_of(gather_index, 8)))
     return HSTU_ERR_UNSUPPORTED;
   prof_begin(HSTU_K_MISC, stream);
-  sl_offsets_kernel<<<1, 1024, 0, stream>>>(seq_offsets, num_targets, B, sub_len, keep_draw,
+  sl_offsets_kernel<<<1, 1024, 0, stream>>>(seq_offsets, num_targets, B, T, sub_len, keep_draw,
                                             new_offsets);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess && B > 0) {
     sl_select_kernel<<<(unsigned)B, kSelThreads, 0, stream>>>(seq_offsets, num_targets, keys,
-                                                               new_offsets, sub_len, gather_index);
+                                                               new_offsets, T, sub_len, gather_index);
     count_launch();
     e = cudaGetLastError();
   }

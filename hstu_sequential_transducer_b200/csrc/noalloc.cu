@@ -16,7 +16,9 @@
 
 namespace {
 
-// Maximum scratch: the work list of up to ~260k (query tile, head) items.
+// Maximum scratch: 2 MiB.  The work list needs 6,400 bytes of counters plus
+// 8 bytes per (128-query tile, head) item, (T / 128 + B + 1) * H items, so it
+// holds up to 261,344 items.
 constexpr size_t kNoAllocScratchBytes = size_t(2) << 20;  // 2 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -26,7 +28,9 @@ void* g_noalloc_ptr[64] = {nullptr};
 
 // Device address of the scratch array on the current device.  Looked up once
 // per device, with that device current; the host-side symbol itself is only
-// a stand-in and must never be passed to a kernel.
+// a stand-in and must never be passed to a kernel.  The cached address stays
+// valid for the life of the device's primary context: a process that resets
+// the device (cudaDeviceReset) must not call this entry point afterwards.
 void* noalloc_scratch(int* err) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
@@ -56,14 +60,13 @@ extern "C" hstu_status hstu_attention_fwd_noalloc(const hstu_config* cfg, const 
                                                   cudaStream_t stream) {
   // The checks of the allocating entry point, run with a zero-sized
   // workspace: they report argument errors without touching the device.
-  size_t need = 0;
-  {
-    const hstu_status st = hstu_attention_fwd(cfg, rab_pos, rab_time, g, seq_offsets, B, T,
-                                              timestamps, num_targets, o_out, nullptr, 0, stream);
-    if (st != HSTU_OK && st != HSTU_ERR_WORKSPACE) return st;
-    if (st == HSTU_OK) return HSTU_OK;  // nothing to compute (empty input)
-    need = hstu_attention_workspace_size(cfg, B, T);
-  }
+  // (a zero-sized workspace always fails its size check, so a well-formed
+  // call comes back with HSTU_ERR_WORKSPACE here).
+  const hstu_status st = hstu_attention_fwd(cfg, rab_pos, rab_time, g, seq_offsets, B, T,
+                                            timestamps, num_targets, o_out, nullptr, 0, stream);
+  if (st != HSTU_ERR_WORKSPACE) return st;
+  if (B == 0 || T == 0) return HSTU_OK;  // nothing to compute; the scratch is not touched
+  const size_t need = hstu_attention_workspace_size(cfg, B, T);
   if (need > kNoAllocScratchBytes) return HSTU_ERR_WORKSPACE;  // beyond the static scratch
   int err = 0;
   void* ws = noalloc_scratch(&err);

@@ -196,11 +196,13 @@ hstu_status hstu_attention_fwd_cached(const hstu_config* cfg, const float* rab_p
  * Meant for processes held to a device-memory budget fixed at start-up, which
  * may not allocate while serving, and for C hosts that own only their input
  * and output buffers.
- *   - Capacity: inputs whose work list exceeds the array (about 260,000
- *     (128-query tile, head) items, i.e. roughly (T / 128 + B) * H <= 262,000)
- *     return HSTU_ERR_WORKSPACE; nothing is launched.
+ *   - Capacity: (floor(T / 128) + B + 1) * H <= 261,344 (128-query tile,
+ *     head) items; larger inputs return HSTU_ERR_WORKSPACE and nothing is
+ *     launched.  Empty inputs (B == 0 or T == 0) return HSTU_OK at once.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the device's primary context: do
+ *     not call this entry point after cudaDeviceReset in the same process.
  *   - It never calls cudaMalloc, cudaFree or any allocating routine.
  *   - Every call on a device shares the same array and rebuilds (and clears)
  *     its contents; calls that can overlap on the GPU (other streams, other
@@ -326,7 +328,10 @@ int64_t hstu_sl_subsequence_length(int64_t max_len, double alpha);
  * row gather_index[r], r < T'.  Build the sampled rows (embeddings,
  * timestamps, ...) with hstu_gather_rows; num_targets is unchanged.
  * Requires T < 2^31; int64 arrays 8-byte and uint32/int32 arrays 4-byte
- * aligned.  Two launches, no synchronisation. */
+ * aligned.  Two launches, no synchronisation.
+ * Malformed offsets (check them with hstu_validate_inputs) give a wrong
+ * sample but no out-of-range access: each sequence's rows are clamped into
+ * [0, T] and no write lands past the T entries of gather_index. */
 hstu_status hstu_stochastic_length(const int64_t* seq_offsets, const int32_t* num_targets,
                                    int32_t B, int64_t T, int64_t sub_len,
                                    const uint32_t* keep_draw, const uint32_t* keys,
@@ -389,6 +394,16 @@ int64_t hstu_launch_count(void);
 #define HSTU_DEVICE_TIMEOUT 0x100u
 #define HSTU_DEVICE_SMEM_ALIGN 0x200u
 hstu_status hstu_device_status(uint32_t* host_out, int32_t clear, cudaStream_t stream);
+
+/* Diagnostic of the bounded-wait path (the pages have no counterpart: this
+ * is this library's failure detection).  Launches one small kernel on
+ * `stream` that waits on an mbarrier nothing ever arrives on, with a limit of
+ * limit_ns nanoseconds (1 .. 100,000,000); the wait runs out, sets
+ * HSTU_DEVICE_TIMEOUT in the device status word and the kernel returns.  It
+ * issues no copy or tensor-core instruction.  d_result (device int32,
+ * nullable) receives 0 when the wait ran out, 1 if it had completed.
+ * Returns HSTU_ERR_INVALID for a limit outside the range, without launching. */
+hstu_status hstu_selftest_wait_timeout(uint64_t limit_ns, int32_t* d_result, cudaStream_t stream);
 
 const char* hstu_status_string(hstu_status s);
 const char* hstu_version(void);

@@ -87,6 +87,7 @@ _SIGS = {
     "hstu_profiler_reset": (None, []),
     "hstu_launch_count": (I64, []),
     "hstu_device_status": (I32, [POINTER(c_uint32), I32, P]),
+    "hstu_selftest_wait_timeout": (I32, [ctypes.c_uint64, P, P]),
     "hstu_status_string": (c_char_p, [I32]),
     "hstu_version": (c_char_p, []),
 }
@@ -460,6 +461,16 @@ def device_status(clear: bool = True, stream=None) -> int:
     _check(lib().hstu_device_status(ctypes.byref(v), 1 if clear else 0, stream_ptr(stream)),
            "hstu_device_status")
     return v.value
+
+
+def selftest_wait_timeout(limit_ns: int, result=None, stream=None):
+    """Launches the library's bounded-wait diagnostic (a wait nothing ends
+    but its limit); the device status word then carries HSTU_DEVICE_TIMEOUT."""
+    _check(lib().hstu_selftest_wait_timeout(int(limit_ns), ptr(result), stream_ptr(stream)),
+           "hstu_selftest_wait_timeout")
+
+
+DEVICE_TIMEOUT, DEVICE_SMEM_ALIGN = 0x100, 0x200
 
 
 def version() -> str:

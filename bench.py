@@ -12,11 +12,18 @@ are synthetic (seeded) and resident in HBM; with N GPUs each rank processes
 its own 64 sequences (weak scaling) and the fp32 gradients are all-reduced
 over NCCL.  Rank 0 prints one JSON line.
 
+With N GPUs each rank processes its own 64 sequences (weak scaling) and each
+layer's fp32 gradients are all-reduced over NCCL as soon as that layer's
+backward has been issued (overlapping the layers below).  --split instead
+shards ONE batch's 64 sequences across the ranks, balanced by n^2 with LPT
+(strong scaling).  The default line also carries `attention_8k`: the two
+attention kernels alone on 16 sequences of exactly 8,192 tokens (H=8,
+dh=128), measured on rank 0 after the timed steps.
+
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on this host's cores (rank 0 only).
 
---attention-8k measures the two attention kernels alone on 16 sequences of
-exactly 8,192 tokens (H=8, dh=128) and prints their TFLOP/s on its own line.
+--attention-8k prints only that attention measurement, on its own line.
 
 --sampler measures the Stochastic Length sampler instead (selection plus the
 gathers of the fp32 rows and timestamps of the training batch, alpha 1.6 by
@@ -92,8 +99,14 @@ def rank_data_seed(rank: int) -> int:
 
 
 def allreduce_grads(flat, dist):
-    """Sums the ranks' gradient buffers in place (one collective per step)."""
+    """Sums the ranks' gradient buffers in place (one collective)."""
     dist.all_reduce(flat)
+
+
+def split_shard(w: W.Workload, rank: int, world: int) -> W.Workload:
+    """Rank `rank`'s part of one batch shared by all ranks: LPT by n^2."""
+    from hstu_sequential_transducer_b200 import dp
+    return W.subset(w, dp.lpt_shards(w.lengths, world)[rank])
 
 
 def max_over_ranks(ms: float, dist, device) -> float:
@@ -104,16 +117,19 @@ def max_over_ranks(ms: float, dist, device) -> float:
     return float(t.item())
 
 
-def make_workload(name, rank, batch=None, layers=None):
+def make_workload(name, rank, batch=None, layers=None, split_world=None):
     """The named workload; `batch` keeps only its first sequences and
     `layers` its first layers (a small case of the same shapes, e.g. for
-    profiler captures)."""
+    profiler captures).  With `split_world`, every rank draws the same batch
+    and keeps its LPT shard of it."""
     if name == "training":
-        w = W.training(data_seed=rank_data_seed(rank))
+        w = W.training(data_seed=rank_data_seed(0 if split_world else rank))
     else:
         w = W.WORKLOADS[name]()
     if batch is not None and batch < w.B:
         w = W.subset(w, list(range(batch)))
+    if split_world:
+        w = split_shard(w, rank, split_world)
     if layers is not None and layers < w.num_layers:
         w.params = w.params[:layers]
         w.num_layers = layers
@@ -308,11 +324,19 @@ def run_ours(args):
         dist.barrier()
     H.lib()
 
-    w = make_workload(args.workload, rank, args.batch, args.layers)
+    from hstu_sequential_transducer_b200 import dp
+    split = bool(args.split) and args.workload == "training"
+    w = make_workload(args.workload, rank, args.batch, args.layers,
+                      split_world=world if split else None)
     dw = S.DeviceWorkload.from_workload(w)
     backward = w.backward
     flops, pairs = workload_flops(w, backward)
     dev = torch.device("cuda", local)
+    # whole-job work: the sum over ranks (ranks' batches differ in size)
+    job = torch.tensor([float(w.T * w.num_layers), float(flops)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(job)
+    job_tokens, job_flops = float(job[0].item()), float(job[1].item())
 
     if args.workload == "mfalcon" and args.batch is None:
         hist, cand = w.meta["history"], w.meta["candidates"]
@@ -321,12 +345,15 @@ def run_ours(args):
             S.mfalcon_score(dw, hist, cand, w.microbatch)
     elif backward:
         ts = S.TrainStep(dw)
+        # each layer's gradients are summed across ranks as soon as its
+        # backward is issued, overlapping the backward of the layers below
+        bk = dp.default_group_bucketing(ts)
 
         def step():
             ts.zero_grads()
-            ts.run()
-            if world > 1:
-                allreduce_grads(ts.flat_grads, dist)
+            ts.run(on_layer_grads=bk.layer_done if bk else None)
+            if bk:
+                bk.wait()
     else:
         def step():
             S.forward_stack(dw)
@@ -367,9 +394,8 @@ def run_ours(args):
             kern[name] = {"launches": n, "total_ms": tot, "avg_ms": tot / n}
     H.profiler_reset()
 
-    tokens = w.T * w.num_layers * world
-    value = tokens / (ms / 1000.0)
-    tflops = flops * world / (ms / 1000.0) / 1e12
+    value = job_tokens / (ms / 1000.0)
+    tflops = job_flops / (ms / 1000.0) / 1e12
     peaks, peak_src = read_peaks()
 
     # dominant kernel and its roofline (algorithmic flops or bytes per launch)
@@ -432,20 +458,33 @@ def run_ours(args):
     # end to end through the public API with host buffers
     e2e = None
     if backward and args.workload == "training" and not args.skip_e2e and args.batch is None:
-        e2e = e2e_training(args, ts, dw, world, dist)
+        e2e = e2e_training(args, ts, dw, world, dist, bk, job_tokens)
+
+    # the attention kernels alone at the length the throughput target names
+    # (rank 0; the other ranks wait at the barrier below)
+    attn8k = None
+    if args.workload == "training" and not args.skip_attention_8k and rank == 0:
+        attn8k = attention8k_measure(args, dev)
+    if world > 1:
+        dist.barrier()
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if split else "weak",
+            "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": f"{args.workload}: {describe(w)}",
-                       "global_batch": w.B * world, "tokens_per_step": w.T * world,
+                       "global_batch": (64 if split else w.B * world),
+                       "tokens_per_step": int(job_tokens) // w.num_layers,
                        "seq_len": int(w.lengths.max()), "max_len": 8192,
                        "layers": w.num_layers, "parallelism": f"dp{world}",
+                       "sharding": ("one batch split across ranks by n^2 (LPT)" if split else
+                                    "each rank its own batch"),
+                       "grad_allreduce": "per-layer buckets, overlapped with the backward",
                        "l2": "inputs larger than L2 (no flush)"},
             "tflops": tflops, "pct_bf16_peak": tflops / peaks.get("bf16_tflops_sustained", 1400.0),
             "roofline": roof, "kernels": kern, "gpu_launches": launches,
-            "clocks": clk, "e2e": e2e}
+            "clocks": clk, "e2e": e2e, "attention_8k": attn8k}
     if rank == 0 and world == 1 and not args.skip_cpu:
         v, desc, threads, _ = oracle_sample(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -458,7 +497,7 @@ def run_ours(args):
     return 0
 
 
-def e2e_training(args, ts, dw, world, dist):
+def e2e_training(args, ts, dw, world, dist, bk, job_tokens):
     """The same training step through the public API, with each step's inputs
     (x, offsets, timestamps, dY; x and dY as bf16) copied from pinned host
     memory and its result (dX, as bf16) read back, all inside the timed
@@ -503,9 +542,9 @@ def e2e_training(args, ts, dw, world, dist):
         dw.offsets, dw.timestamps, dw.dy = off, tst, dy
         ts.acts[0] = x
         ts.zero_grads()
-        dx = ts.run()
-        if world > 1:
-            allreduce_grads(ts.flat_grads, dist)
+        dx = ts.run(on_layer_grads=bk.layer_done if bk else None)
+        if bk:
+            bk.wait()
         comp.wait_event(drained[s])
         stage[s].copy_(dx)
         consumed[s].record(comp)
@@ -534,7 +573,7 @@ def e2e_training(args, ts, dw, world, dist):
     if world > 1:
         ms = max_over_ranks(ms, dist, dev)
     dw.x, dw.offsets, dw.timestamps, dw.dy, ts.acts[0] = saved_inputs
-    return {"value": w.T * w.num_layers * world / (ms / 1000.0), "unit": "tokens/s",
+    return {"value": job_tokens / (ms / 1000.0), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms,
             "copies": "second stream, double-buffered: next step's inputs uploaded and the "
                       "previous step's dX downloaded while a step computes"}
@@ -793,14 +832,50 @@ def run_attention8k(args):
     build.build()
     H.lib()
     dev = torch.device("cuda", local)
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = H.launch_count()
+    m = attention8k_measure(args, dev)
+    launches = H.launch_count() - launches0
+    clk = clocks.stop()
+    peaks, peak_src = read_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    line = {"metric": ATTN8K_METRIC, "value": m["tflops"], "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": m["workload"], "tokens_per_step": m["tokens"],
+                       "l2": "inputs larger than L2 (no flush)", "parallelism": "dp1"},
+            "attn_fwd": m["attn_fwd"], "attn_bwd": m["attn_bwd"],
+            "roofline": {"kernel": "attn_bwd", "bound": "tensor", "achieved": m["attn_bwd"]["tflops"],
+                         "peak": peak, "unit": "TFLOP/s", "frac": m["attn_bwd"]["frac"],
+                         "traffic": None, "peak_source": f"{peak_src} (bf16_tflops_sustained)",
+                         "work_per_launch": m["attn_bwd"]["flops"]},
+            "gpu_launches": launches, "clocks": clk, "e2e": None}
+    if not args.skip_cpu:
+        v, desc = attn8k_oracle(args.cpu_budget)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def attention8k_measure(args, dev):
+    """The attention forward and backward kernels alone on B sequences of
+    exactly 8,192 tokens (d = 1,024, H = 8, dh = 128, causal, position and time
+    rab, N = 8,192), each timed with CUDA events around its launch on the
+    current stream; median over the timed steps."""
+    import torch
+
+    from hstu_sequential_transducer_b200 import hstu as H
     B, n, d, nh = (args.batch or 16), 8192, 1024, 8
     T = B * n
-    rng = np.random.default_rng(7 + rank)
+    rng = np.random.default_rng(7)
     cfg = H.make_config(d, nh, 8192.0, H.HSTU_BF16, 32, 32, 8192)
     offs = torch.arange(B + 1, dtype=torch.int64, device=dev) * n
     ts = torch.from_numpy(W.draw_timestamps(rng, [n] * B)).to(dev)
     gen = torch.Generator(device=dev)
-    gen.manual_seed(11 + rank)
+    gen.manual_seed(11)
     g = (torch.randn(T, 4 * d, device=dev, generator=gen) * 0.5).to(torch.bfloat16)
     pre = torch.randn(T, 4 * d, device=dev, generator=gen).to(torch.bfloat16)
     dout = torch.randn(T, d, device=dev, generator=gen).to(torch.bfloat16)
@@ -825,48 +900,31 @@ def run_attention8k(args):
             e[2].record()
             ev.append(e)
 
-    for _ in range(args.warmup):
+    for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local)
-    clocks.start()
-    launches0 = H.launch_count()
-    torch.cuda.synchronize()
+    steps = max(args.steps, 5)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
+    for _ in range(steps):
         step(timed=True)
     e1.record()
     torch.cuda.synchronize()
-    launches = H.launch_count() - launches0
-    clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = e0.elapsed_time(e1) / steps
     fwd_ms = float(np.median([a.elapsed_time(b) for a, b, _ in ev]))
     bwd_ms = float(np.median([b.elapsed_time(c) for _, b, c in ev]))
     peaks, peak_src = read_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     fwd_tf, bwd_tf = f_fwd / fwd_ms / 1e9, f_bwd / bwd_ms / 1e9
-    line = {"metric": ATTN8K_METRIC, "value": (f_fwd + f_bwd) / ms / 1e9, "unit": "TFLOP/s",
-            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": f"attention at 8192: B={B} sequences of 8,192 tokens, d=1024, "
-                                   "H=8, dh=128, causal, 32+32 rab buckets, N=8192",
-                       "tokens_per_step": T, "l2": "inputs larger than L2 (no flush)",
-                       "parallelism": "dp1"},
-            "attn_fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
-            "attn_bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
-            "roofline": {"kernel": "attn_bwd", "bound": "tensor", "achieved": bwd_tf, "peak": peak,
-                         "unit": "TFLOP/s", "frac": bwd_tf / peak, "traffic": None,
-                         "peak_source": f"{peak_src} (bf16_tflops_sustained)",
-                         "work_per_launch": f_bwd},
-            "gpu_launches": launches, "clocks": clk, "e2e": None}
-    if not args.skip_cpu:
-        v, desc = attn8k_oracle(args.cpu_budget)
-        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
-                                "kind": "oracle", "sample": desc}
-    print(json.dumps(line), flush=True)
-    return 0
+    out = {"workload": f"attention at 8192: B={B} sequences of 8,192 tokens, d=1024, H=8, dh=128, "
+                       "causal, 32+32 rab buckets, N=8192",
+           "tokens": T, "steps": steps, "ms": ms, "tflops": (f_fwd + f_bwd) / ms / 1e9,
+           "attn_fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak, "flops": f_fwd},
+           "attn_bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak, "flops": f_bwd},
+           "peak": peak, "peak_source": f"{peak_src} (bf16_tflops_sustained)"}
+    del g, pre, dout, o, dpre
+    torch.cuda.empty_cache()
+    return out
 
 
 def main(argv=None):
@@ -888,6 +946,10 @@ def main(argv=None):
     ap.add_argument("--alpha", type=float, default=1.6)
     ap.add_argument("--attention-8k", action="store_true",
                     help="measure the attention kernels alone on 16 sequences of 8,192 tokens")
+    ap.add_argument("--skip-attention-8k", action="store_true",
+                    help="leave the attention_8k measurement out of the default line")
+    ap.add_argument("--split", action="store_true",
+                    help="shard one training batch across the ranks (LPT by n^2; strong scaling)")
     args = ap.parse_args(argv)
     if args.attention_8k:
         return run_attention8k(args)

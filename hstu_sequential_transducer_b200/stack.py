@@ -97,21 +97,29 @@ class TrainStep:
                     total += (t.numel() + 63) // 64 * 64
         self.flat_grads = torch.zeros(max(total, 1), dtype=torch.float32, device=dev)
         self.grads = []
+        # layer i's gradients occupy elements [sum(sizes[:i]), sum(sizes[:i+1]))
+        # of the flat buffer: one bucket per layer for an overlapped all-reduce
+        self.layer_grad_sizes = []
         o = 0
         for w in dw.layers:
             gb = H.LayerGradBufs()
+            o0 = o
             for n, gn in zip(names, gnames):
                 t = getattr(w, n)
                 if t is not None:
                     setattr(gb, gn, self.flat_grads[o:o + t.numel()].view(t.shape))
                     o += (t.numel() + 63) // 64 * 64
             self.grads.append(gb)
+            self.layer_grad_sizes.append(o - o0)
 
     def zero_grads(self):
         self.flat_grads.zero_()
 
-    def run(self, dy=None, stream=None):
-        """Forward (keeping activations) then backward from dy; returns dX."""
+    def run(self, dy=None, stream=None, on_layer_grads=None):
+        """Forward (keeping activations) then backward from dy; returns dX.
+        on_layer_grads(i), when given, is called right after layer i's
+        backward has been issued (layers in reverse order), e.g. to start the
+        all-reduce of that layer's gradients."""
         dw = self.dw
         for i, w in enumerate(dw.layers):
             H.fwd(dw.cfg, w, self.acts[i], dw.offsets, dw.timestamps, dw.num_targets,
@@ -121,6 +129,8 @@ class TrainStep:
             out = self.gbuf[i % 2]
             H.bwd(dw.cfg, dw.layers[i], self.acts[i], g, self.saved[i], dw.offsets, dw.timestamps,
                   dw.num_targets, dx=out, grads=self.grads[i], stream=stream)
+            if on_layer_grads is not None:
+                on_layer_grads(i)
             g = out
         return g
 
@@ -129,11 +139,23 @@ class TrainStep:
         return self.acts[-1]
 
 
+def _gather(src, rows: np.ndarray, out=None):
+    """out[r] = src[rows[r]] through the library's row gather (the index and
+    the row count are uploaded once per call; no PyTorch indexing)."""
+    dev = src.device
+    idx = torch.from_numpy(np.ascontiguousarray(rows, dtype=np.int64)).to(dev)
+    count = torch.tensor([len(rows)], dtype=torch.int64, device=dev)
+    if out is None:
+        out = torch.empty((len(rows),) + tuple(src.shape[1:]), dtype=src.dtype, device=dev)
+    return H.gather_rows(src, idx, count, out)
+
+
 def mfalcon_score(dw: DeviceWorkload, history: int, candidates: int, microbatch: int, stream=None):
     """M-FALCON scoring of a workload whose users are `history` tokens followed
     by `candidates` tokens: one history pass caching each layer's V|K, then the
     candidates in microbatches against the cache.  Returns (y_hist, y_cand)
-    with candidate rows in input order."""
+    with candidate rows in input order.  Row selection and reordering run in
+    the library's gather kernel."""
     w = dw.w
     B = w.B
     dev = dw.x.device
@@ -142,9 +164,8 @@ def mfalcon_score(dw: DeviceWorkload, history: int, candidates: int, microbatch:
     assert np.all(w.lengths == n)
     base = np.arange(B) * n
     hist_rows = (base[:, None] + np.arange(history)[None, :]).reshape(-1)
-    hist_rows_t = torch.from_numpy(hist_rows).to(dev)
-    x_hist = dw.x.index_select(0, hist_rows_t)
-    ts_hist = dw.timestamps.index_select(0, hist_rows_t)
+    x_hist = _gather(dw.x, hist_rows)
+    ts_hist = _gather(dw.timestamps, hist_rows)
     hist_off = torch.arange(B + 1, dtype=torch.int64, device=dev) * history
     caches = []
     y = x_hist
@@ -153,18 +174,25 @@ def mfalcon_score(dw: DeviceWorkload, history: int, candidates: int, microbatch:
         y = H.fwd(dw.cfg, lw, y, hist_off, ts_hist, None, kv_out=kv, stream=stream)
         caches.append(kv)
     y_hist = y
-    y_cand = torch.empty(B * candidates, d, dtype=dw.x.dtype, device=dev)
+    # microbatch k writes its B * mb_k rows (user-major) into its own slice of
+    # ybuf; one gather then puts every candidate back in input order
+    ybuf = torch.empty(B * candidates, d, dtype=dw.x.dtype, device=dev)
+    src_rows = np.empty((B, candidates), dtype=np.int64)
+    done = 0
     for k0 in range(0, candidates, microbatch):
         mb = min(microbatch, candidates - k0)
         rows = (base[:, None] + history + k0 + np.arange(mb)[None, :]).reshape(-1)
-        rows_t = torch.from_numpy(rows).to(dev)
-        xc = dw.x.index_select(0, rows_t)
-        tc = dw.timestamps.index_select(0, rows_t)
+        xc = _gather(dw.x, rows)
+        tc = _gather(dw.timestamps, rows)
         coff = torch.arange(B + 1, dtype=torch.int64, device=dev) * mb
+        out = ybuf[done:done + B * mb]
         for li, lw in enumerate(dw.layers):
-            xc = H.fwd_cached(dw.cfg, lw, xc, coff, tc, caches[li], hist_off, ts_hist, stream=stream)
-        out_rows = (np.arange(B)[:, None] * candidates + k0 + np.arange(mb)[None, :]).reshape(-1)
-        y_cand[torch.from_numpy(out_rows).to(dev)] = xc
+            last = li == len(dw.layers) - 1
+            xc = H.fwd_cached(dw.cfg, lw, xc, coff, tc, caches[li], hist_off, ts_hist,
+                              y=out if last else None, stream=stream)
+        src_rows[:, k0:k0 + mb] = done + np.arange(B)[:, None] * mb + np.arange(mb)[None, :]
+        done += B * mb
+    y_cand = _gather(ybuf, src_rows.reshape(-1))
     return y_hist, y_cand
 
 

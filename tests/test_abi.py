@@ -139,3 +139,18 @@ def test_sl_binding_rejects_wrong_dtypes(L):
     with pytest.raises(ValueError):
         H.stochastic_length(offs, None, 5, torch.zeros(3, dtype=torch.int32),
                             torch.zeros(4, dtype=torch.int32))
+
+
+@pytest.mark.parametrize("d,nh", [(512, 4), (1024, 8)])
+def test_saved_activation_budget_within_14d(L, d, nh):
+    """The HSTU walkthrough ("Gating instead of a separate FFN") puts an HSTU
+    layer's saved activation state at 14d bf16 values per token (against 33d
+    for a Transformer layer).  The layer's saved block (Pre and G = SiLU(Pre)
+    in bf16, O in fp32, Z, the bf16 copy of the residual input, the LayerNorm
+    statistics) stays within that: 24d + 8 bytes = 12d + 4 bf16 values."""
+    T = 1_000_000
+    c = H.make_config(d, nh, 8192.0, H.HSTU_BF16)
+    off = H.saved_layout(c, T)
+    per_token = off[-1] / T
+    assert per_token <= 24 * d + 8 + 1e-3 * d
+    assert per_token <= 2 * 14 * d

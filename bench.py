@@ -846,7 +846,8 @@ def run_attention8k(args):
             "data": "synthetic",
             "config": {"workload": m["workload"], "tokens_per_step": m["tokens"],
                        "l2": "inputs larger than L2 (no flush)", "parallelism": "dp1"},
-            "attn_fwd": m["attn_fwd"], "attn_bwd": m["attn_bwd"],
+            "attn_fwd": m["attn_fwd"], "attn_bwd": m["attn_bwd"], "softmax_fwd": m["softmax_fwd"],
+            "pointwise_fwd_speedup_over_softmax": m["pointwise_fwd_speedup_over_softmax"],
             "roofline": {"kernel": "attn_bwd", "bound": "tensor", "achieved": m["attn_bwd"]["tflops"],
                          "peak": peak, "unit": "TFLOP/s", "frac": m["attn_bwd"]["frac"],
                          "traffic": None, "peak_source": f"{peak_src} (bf16_tflops_sustained)",
@@ -889,7 +890,7 @@ def attention8k_measure(args, dev):
     ev = []
 
     def step(timed=False):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if timed else None
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if timed else None
         if timed:
             e[0].record()
         H.attention_fwd(cfg, rab_pos, rab_time, g, offs, ts, None, o)
@@ -898,6 +899,11 @@ def attention8k_measure(args, dev):
         H.attention_bwd(cfg, rab_pos, rab_time, g, pre, dout, offs, ts, None, dpre, drp, drt)
         if timed:
             e[2].record()
+        # the softmax comparison kernel on the same inputs (not part of the step's
+        # HSTU work: timed on its own and reported beside the pointwise forward)
+        H.softmax_attention_fwd(cfg, rab_pos, rab_time, g, offs, ts, None, o)
+        if timed:
+            e[3].record()
             ev.append(e)
 
     for _ in range(max(args.warmup, 3)):
@@ -910,9 +916,10 @@ def attention8k_measure(args, dev):
         step(timed=True)
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    fwd_ms = float(np.median([a.elapsed_time(b) for a, b, _ in ev]))
-    bwd_ms = float(np.median([b.elapsed_time(c) for _, b, c in ev]))
+    fwd_ms = float(np.median([a.elapsed_time(b) for a, b, _, _ in ev]))
+    bwd_ms = float(np.median([b.elapsed_time(c) for _, b, c, _ in ev]))
+    smx_ms = float(np.median([c.elapsed_time(d) for _, _, c, d in ev]))
+    ms = e0.elapsed_time(e1) / steps - smx_ms
     peaks, peak_src = read_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     fwd_tf, bwd_tf = f_fwd / fwd_ms / 1e9, f_bwd / bwd_ms / 1e9
@@ -921,6 +928,10 @@ def attention8k_measure(args, dev):
            "tokens": T, "steps": steps, "ms": ms, "tflops": (f_fwd + f_bwd) / ms / 1e9,
            "attn_fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak, "flops": f_fwd},
            "attn_bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak, "flops": f_bwd},
+           "softmax_fwd": {"ms": smx_ms, "tflops": f_fwd / smx_ms / 1e9,
+                           "frac": f_fwd / smx_ms / 1e9 / peak, "flops": f_fwd,
+                           "what": "softmax comparison kernel, same score, mask and tiling"},
+           "pointwise_fwd_speedup_over_softmax": smx_ms / fwd_ms,
            "peak": peak, "peak_source": f"{peak_src} (bf16_tflops_sustained)"}
     del g, pre, dout, o, dpre
     torch.cuda.empty_cache()

@@ -550,6 +550,31 @@ hstu_status hstu_attention_fwd(const hstu_config* cfg, const float* rab_pos, con
   return do_attention_fwd(cfg, a, workspace, ws_bytes, stream, HSTU_K_ATTN_FWD);
 }
 
+hstu_status hstu_softmax_attention_fwd(const hstu_config* cfg, const float* rab_pos,
+                                       const float* rab_time, const void* g,
+                                       const int64_t* seq_offsets, int32_t B, int64_t T,
+                                       const int64_t* timestamps, const int32_t* num_targets,
+                                       void* o_out, void* workspace, size_t ws_bytes,
+                                       cudaStream_t stream) {
+  HSTU_TRY(check_cfg(cfg));
+  HSTU_TRY(check_jagged(seq_offsets, B, T, timestamps, num_targets));
+  HSTU_TRY(need(g, T));
+  HSTU_TRY(need(o_out, T));
+  HSTU_TRY(meta(rab_pos, rab_pos ? 1 : 0, 4));
+  HSTU_TRY(meta(rab_time, rab_time ? 1 : 0, 4));
+  const size_t need_ws = attention_fwd_ws(B, T, cfg->num_heads, cfg->max_seq_len);
+  if (ws_bytes < need_ws) return HSTU_ERR_WORKSPACE;
+  if (need_ws > 0) HSTU_TRY(need(workspace, 1));
+  if (T == 0 || B == 0) return HSTU_OK;
+  AttnArgs a = full_attn_args(cfg, rab_pos, rab_time, g, seq_offsets, B, T, timestamps,
+                              num_targets, o_out);
+  if (!softmax_fwd_tc_supported(cfg->dtype, a)) return HSTU_ERR_UNSUPPORTED;
+  prof_begin(HSTU_K_SOFTMAX, stream);
+  cudaError_t e = softmax_fwd_tc(a, workspace, device_status(), stream);
+  prof_end(HSTU_K_SOFTMAX, stream);
+  return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
 hstu_status hstu_attention_fwd_cached(const hstu_config* cfg, const float* rab_pos,
                                       const float* rab_time, const void* cand_g,
                                       const int64_t* cand_offsets, int32_t B, int64_t Tc,

@@ -40,6 +40,7 @@
 // (diagonal, tails, candidates' near keys) evaluate buckets per element.
 #include <cuda.h>
 
+#include "attn_sched.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -47,25 +48,6 @@
 namespace hstu {
 
 using namespace tc;
-
-// ---------------------------------------------------------------------------
-// Work list: items sorted by descending number of key tiles
-// ---------------------------------------------------------------------------
-struct AttnItem {
-  int32_t b;
-  int16_t qt;
-  int16_t h;
-};
-
-constexpr int kTile = 128;
-constexpr int kMaxCost = 514;  // key tiles per item, 65536 / 128 + 2
-
-struct SchedWs {
-  int32_t* hist;     // [kMaxCost]
-  int32_t* cursor;   // [kMaxCost]
-  int32_t* total;    // [1]
-  AttnItem* items;   // [max_items]
-};
 
 size_t attn_sched_bytes(int B, int64_t Tq, int H) {
   const size_t max_items = ((size_t)(Tq / kTile) + (size_t)B + 1) * (size_t)H;
@@ -79,35 +61,6 @@ SchedWs sched_ws(void* ws) {
   s.total = s.cursor + kMaxCost;
   s.items = reinterpret_cast<AttnItem*>(static_cast<char*>(ws) + align_up(3 * kMaxCost * sizeof(int32_t), 256));
   return s;
-}
-
-// Key tiles an item needs, and the item's geometry.
-struct SeqGeom {
-  int64_t qs, ks;   // first query row, first key row
-  int nq, hlen;     // queries; keys visible to candidates (= history length)
-  int qbase;        // position of query 0
-};
-
-__device__ __forceinline__ SeqGeom seq_geom(const AttnArgs& a, int b) {
-  SeqGeom g;
-  g.qs = a.q_offsets[b];
-  g.nq = (int)(a.q_offsets[b + 1] - g.qs);
-  g.ks = a.kv_offsets[b];
-  const int nkv = (int)(a.kv_offsets[b + 1] - g.ks);
-  if (a.cached) {
-    g.hlen = nkv;
-    g.qbase = nkv;
-  } else {
-    const int m = a.num_targets ? a.num_targets[b] : 0;
-    g.hlen = min(max(g.nq - m, 0), g.nq);
-    g.qbase = 0;
-  }
-  return g;
-}
-
-__device__ __forceinline__ int item_kend(const SeqGeom& g, int qt) {
-  const int rows = min(kTile, g.nq - qt * kTile);
-  return min(g.hlen, g.qbase + qt * kTile + rows);
 }
 
 __global__ void sched_count_kernel(AttnArgs a, SchedWs w) {

@@ -99,6 +99,9 @@ size_t attn_bwd_sched_bytes(int B, int64_t T, int H);
 bool attention_bwd_tc_supported(int dtype, const AttnBwdArgs& a);
 cudaError_t attention_bwd_tc(const AttnBwdArgs& a, void* ws, uint32_t* status, cudaStream_t s);
 cudaError_t attention_bwd_self_simt(int dtype, const AttnBwdArgs& a, cudaStream_t s);
+// Softmax comparison attention (same score, buckets and mask; bf16, dh 64/128).
+bool softmax_fwd_tc_supported(int dtype, const AttnArgs& a);
+cudaError_t softmax_fwd_tc(const AttnArgs& a, void* ws, uint32_t* status, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // LayerNorm (.) U epilogue

@@ -21,9 +21,9 @@ LIB_PATH = os.path.join(_HERE, "libhstu.so")
 HSTU_F32, HSTU_BF16 = 0, 1
 SAVED_PRE, SAVED_G, SAVED_O, SAVED_Z, SAVED_MEAN, SAVED_RSTD, SAVED_XLOW, SAVED_COUNT = range(8)
 K_PROJ_IN, K_ATTN_FWD, K_LN_FWD, K_PROJ_OUT, K_PROJ_OUT_BWD, K_LN_BWD, K_ATTN_BWD, \
-    K_PROJ_IN_BWD, K_ATTN_CACHED, K_MISC, K_COUNT = range(11)
+    K_PROJ_IN_BWD, K_ATTN_CACHED, K_MISC, K_SOFTMAX, K_COUNT = range(12)
 KERNEL_NAMES = ["proj_in", "attn_fwd", "ln_fwd", "proj_out", "proj_out_bwd", "ln_bwd",
-                "attn_bwd", "proj_in_bwd", "attn_cached", "misc"]
+                "attn_bwd", "proj_in_bwd", "attn_cached", "misc", "softmax_fwd"]
 
 FLAG_OFFSETS_START, FLAG_OFFSETS_ORDER, FLAG_OFFSETS_END = 0x1, 0x2, 0x4
 FLAG_SEQ_TOO_LONG, FLAG_TARGETS_RANGE, FLAG_TIME_ORDER = 0x8, 0x10, 0x20
@@ -67,6 +67,7 @@ _SIGS = {
     "hstu_attention_fwd": (I32, [_CP, P, P, P, P, I32, I64, P, P, P, P, S, P]),
     "hstu_attention_fwd_cached": (I32, [_CP, P, P, P, P, I32, I64, P, P, P, I64, P, P, P, S, P]),
     "hstu_attention_workspace_size": (S, [_CP, I32, I64]),
+    "hstu_softmax_attention_fwd": (I32, [_CP, P, P, P, P, I32, I64, P, P, P, P, S, P]),
     "hstu_attention_fwd_noalloc": (I32, [_CP, P, P, P, P, I32, I64, P, P, P, P]),
     "hstu_ln_gate_fwd": (I32, [_CP, P, P, P, P, I64, P, P, P, P]),
     "hstu_proj_out_fwd": (I32, [_CP, P, P, P, P, I64, P, P]),
@@ -254,6 +255,18 @@ def attention_fwd(cfg, rab_pos, rab_time, g, offsets, timestamps, num_targets, o
                                     ptr(offsets), B, T, ptr(timestamps), ptr(num_targets),
                                     ptr(o_out), ptr(ws), ws.numel(), stream_ptr(stream)),
            "hstu_attention_fwd")
+
+
+def softmax_attention_fwd(cfg, rab_pos, rab_time, g, offsets, timestamps, num_targets, o_out,
+                          stream=None):
+    """The softmax comparison attention (same score and mask, softmax weights)."""
+    B, T = offsets.numel() - 1, g.shape[0]
+    n = lib().hstu_attention_workspace_size(ctypes.byref(cfg), B, T)
+    ws = workspace(n, g.device, "attn")
+    _check(lib().hstu_softmax_attention_fwd(ctypes.byref(cfg), ptr(rab_pos), ptr(rab_time), ptr(g),
+                                            ptr(offsets), B, T, ptr(timestamps), ptr(num_targets),
+                                            ptr(o_out), ptr(ws), ws.numel(), stream_ptr(stream)),
+           "hstu_softmax_attention_fwd")
 
 
 def attention_fwd_noalloc(cfg, rab_pos, rab_time, g, offsets, timestamps, num_targets, o_out,

@@ -213,6 +213,23 @@ hstu_status hstu_attention_fwd_noalloc(const hstu_config* cfg, const float* rab_
                                        const int64_t* timestamps, const int32_t* num_targets,
                                        void* o_out, cudaStream_t stream);
 
+/* Softmax comparison attention (HSTU walkthrough, "No sequence-wise
+ * softmax": HSTU's pointwise SiLU aggregation against the softmax attention of
+ * a standard Transformer, which the paper's speed claim at length 8,192 is
+ * measured against).  Same arguments, layouts, workspace and errors as
+ * hstu_attention_fwd, and the same score S_h(i, j) = Q_h(i).K_h(j) +
+ * rab_pos[h][bp] + rab_time[h][bt] (no 1/sqrt(dh)) and mask; the weights are
+ * softmax_j(S_h(i, j)) over each query's allowed keys instead of
+ * SiLU(S_h(i, j)) / N (norm_N is not used).  o_out [T][d] fp32.  Tensor cores
+ * only: bf16 with head_dim 64 or 128, else HSTU_ERR_UNSUPPORTED.  For timing
+ * against the pointwise kernel; it is not part of the layer. */
+hstu_status hstu_softmax_attention_fwd(const hstu_config* cfg, const float* rab_pos,
+                                       const float* rab_time, const void* g,
+                                       const int64_t* seq_offsets, int32_t B, int64_t T,
+                                       const int64_t* timestamps, const int32_t* num_targets,
+                                       void* o_out, void* workspace, size_t ws_bytes,
+                                       cudaStream_t stream);
+
 /* Bytes of workspace the attention entry points need. Host only. */
 size_t hstu_attention_workspace_size(const hstu_config* cfg, int32_t B, int64_t T);
 
@@ -372,7 +389,7 @@ hstu_status hstu_validate_inputs(const int64_t* seq_offsets, int32_t B, int64_t 
 typedef enum {
   HSTU_K_PROJ_IN = 0, HSTU_K_ATTN_FWD = 1, HSTU_K_LN_FWD = 2, HSTU_K_PROJ_OUT = 3,
   HSTU_K_PROJ_OUT_BWD = 4, HSTU_K_LN_BWD = 5, HSTU_K_ATTN_BWD = 6, HSTU_K_PROJ_IN_BWD = 7,
-  HSTU_K_ATTN_CACHED = 8, HSTU_K_MISC = 9, HSTU_K_COUNT = 10
+  HSTU_K_ATTN_CACHED = 8, HSTU_K_MISC = 9, HSTU_K_SOFTMAX = 10, HSTU_K_COUNT = 11
 } hstu_kernel_id;
 
 void hstu_profiler_enable(int32_t on);

@@ -248,8 +248,14 @@ __global__ void __launch_bounds__(352, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const FwdParams P) {
   using C = FwdCfg<DH>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // the base stays the __shared__ array itself, so that every access
+  // through it compiles to a shared-memory (not a generic) access
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {              // uniform over the block: all threads leave
+    if (threadIdx.x == 0 && P.status) atomicOr(P.status, kStatusSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::TILE_BYTES;                      // K_STAGES tiles
   uint8_t* sV = sK + C::K_STAGES * C::TILE_BYTES;        // V_STAGES tiles

@@ -37,7 +37,9 @@
 // non-decreasing), changes at no more than two breakpoints, found by binary
 // search over the tile's timestamps once per row and tile.  Rows of a warp
 // that all qualify take that path (a few compares per element); the others
-// (diagonal, tails, candidates' near keys) evaluate buckets per element.
+// (diagonal, tails, candidates' near keys) evaluate buckets per element, in a
+// rolled loop over eight columns at a time (small code for a path that runs
+// once or twice per item).
 #include <cuda.h>
 
 #include "attn_sched.cuh"
@@ -155,20 +157,6 @@ __device__ __forceinline__ float silu_half(float h) {
 
 __device__ __forceinline__ int time_bucket32(long long dt, int Bt) {
   return dt <= 0 ? 0 : min(64 - __clzll(dt), Bt - 1);
-}
-
-__device__ __forceinline__ int time_bucket_lo(uint32_t tq_lo, uint32_t tk_lo, int Bt) {
-  const int dt = (int)(tq_lo - tk_lo);
-  return dt <= 0 ? 0 : min(32 - __clz(dt), Bt - 1);
-}
-
-// Number of the 32 non-decreasing values cts[] that are <= tau.
-__device__ __forceinline__ int count_le32(const long long* cts, long long tau) {
-  int lo = 0;
-#pragma unroll
-  for (int step = 16; step >= 1; step >>= 1)
-    if (cts[lo + step - 1] <= tau) lo += step;
-  return lo + (cts[lo] <= tau ? 1 : 0);
 }
 
 // Number of the 128 non-decreasing values cts[] that are <= tau.
@@ -573,80 +561,38 @@ __global__ void __launch_bounds__(352, 1)
           else if (nbw == 1) act_tile_fast<1>(sbuf, pbuf, hb, p, hd);
           else act_tile_fast<2>(sbuf, pbuf, hb, p, hd);
         } else {
-          const int last = max(min(kTile, kend - k0) - 1, 0);
-          const long long g_hi = tq - kts[0], g_lo = tq - kts[last];
-          const bool gap32 = __all_sync(0xffffffffu, !rvalid || (g_hi < 0x7fffffffLL && g_lo > -0x7fffffffLL));
-          const uint32_t tq_lo = (uint32_t)(unsigned long long)tq;
-          const uint32_t* kts_lo = reinterpret_cast<const uint32_t*>(kts);
+          // diagonal, partial and near tiles, once or twice per item: every
+          // element on its own, eight columns per pass of a rolled loop.  The
+          // code stays small, so that between two such tiles the fast path
+          // does not push it out of the instruction cache.
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            const int c0 = c * 32;
-            uint32_t sv[32], pk[16];
-            tmem_ld32(sbuf + c0, sv);
-            const int j0 = k0 + c0;
-            const bool masked = !rvalid || j0 >= kend || (!cand && j0 > qpos);
-            const bool visible = rvalid && j0 + 31 < kend && (cand || j0 + 31 <= qpos);
-            const bool cfar = qp_clamped - (j0 + 31) >= a.P - 1;
-            int cb_lo = 0, cnb = 3;
-            if (visible && cfar) {
-              cb_lo = time_bucket32(tq - kts[c0 + 31], a.Bt);
-              cnb = time_bucket32(tq - kts[c0], a.Bt) - cb_lo;
-            }
-            const bool all_masked = __all_sync(0xffffffffu, masked);
-            const bool cfast = __all_sync(0xffffffffu, visible && cfar && cnb <= 2);
+          for (int c8 = 0; c8 < kTile / 8; ++c8) {
+            const int col0 = c8 * 8;
+            uint32_t sv[8], pk[4];
+            tmem_ld8(sbuf + col0, sv);
+            const int j0 = k0 + col0;
+            const bool all_masked = __all_sync(0xffffffffu, !rvalid || j0 >= kend || (!cand && j0 > qpos));
             tmem_ld_wait();
             if (all_masked) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) pk[e] = 0u;
-            } else if (cfast) {
-              const int nbw = __reduce_max_sync(0xffffffffu, (unsigned)cnb);
-              int p[2] = {0, 0};
-              float hd[2] = {0.f, 0.f};
-#pragma unroll
-              for (int k = 0; k < 2; ++k)
-                if (k < cnb) {
-                  const int b = cb_lo + 1 + k;
-                  p[k] = c0 + count_le32(kts + c0, tq - (1LL << (b - 1)));
-                  hd[k] = 0.5f * (rab[32 + b] - rab[32 + b - 1]);
-                }
-              const float hb = 0.5f * (rp_far + rab[32 + cb_lo]);
-              if (nbw == 0) act_chunk_fast<0>(sv, c0, hb, p, hd, pk);
-              else if (nbw == 1) act_chunk_fast<1>(sv, c0, hb, p, hd, pk);
-              else act_chunk_fast<2>(sv, c0, hb, p, hd, pk);
-            } else if (gap32) {
-#pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                float y[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                  const int col = c * 32 + e + u;
-                  const int jk = k0 + col;
-                  const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
-                  const int bp = min(max(qp_clamped - jk, 0), a.P - 1);
-                  const int bt = time_bucket_lo(tq_lo, kts_lo[2 * col], a.Bt);
-                  const float h = 0.5f * (__uint_as_float(sv[e + u]) + rab[bp] + rab[32 + bt]);
-                  y[u] = ok ? silu_half(h) : 0.f;
-                }
-                pk[e / 2] = pack_bf16(y[0], y[1]);
-              }
+              for (int e = 0; e < 4; ++e) pk[e] = 0u;
             } else {
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) {
+              for (int e = 0; e < 8; e += 2) {
                 float y[2];
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                  const int col = c * 32 + e + u;
-                  const int jk = k0 + col;
+                  const int jk = j0 + e + u;
                   const bool ok = rvalid && jk < kend && (cand || jk <= qpos);
                   const int bp = min(max(qp_clamped - jk, 0), a.P - 1);
-                  const int bt = time_bucket32(tq - kts[col], a.Bt);
+                  const int bt = time_bucket32(tq - kts[col0 + e + u], a.Bt);
                   const float h = 0.5f * (__uint_as_float(sv[e + u]) + rab[bp] + rab[32 + bt]);
                   y[u] = ok ? silu_half(h) : 0.f;
                 }
                 pk[e / 2] = pack_bf16(y[0], y[1]);
               }
             }
-            tmem_st16(pbuf + c * 16, pk);
+            tmem_st4(pbuf + c8 * 4, pk);
           }
         }
         tmem_st_wait();

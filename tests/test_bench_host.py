@@ -55,3 +55,24 @@ def test_attention_8k_reference_line():
     d = run_line(["--attention-8k", "--impl", "reference", "--cpu-budget", "0.1"])
     assert KEYS <= set(d) and d["impl"] == "reference" and d["unit"] == "TFLOP/s"
     assert d["value"] > 0
+
+
+def test_split_shards_partition_one_batch():
+    """--split: every rank draws the same batch and keeps its LPT share; the
+    shares partition the batch's sequences and tokens."""
+    w = W.custom([9, 3, 12, 5, 7, 2, 30], d=16, H=2, layers=1, seed=4)
+    for world in (1, 2, 3):
+        parts = [bench.split_shard(w, r, world) for r in range(world)]
+        assert sum(p.T for p in parts) == w.T
+        assert sum(p.B for p in parts) == w.B
+        rows = np.concatenate([p.x for p in parts])
+        assert sorted(map(tuple, rows.round(6))) == sorted(map(tuple, w.x.round(6)))
+
+
+def test_training_reference_line():
+    """The default reference arm (the oracle on a bounded sample) prints one
+    JSON line with the base contract's keys."""
+    d = run_line(["--impl", "reference", "--batch", "2", "--layers", "1", "--steps", "1",
+                  "--warmup", "0"])
+    assert KEYS <= set(d) and d["impl"] == "reference" and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0

@@ -452,11 +452,14 @@ __global__ void __launch_bounds__(352, 1)
             const int stage = (int)(nj % C::K_STAGES);
             if (!mbar_wait(&k_full[stage], (nj / C::K_STAGES) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t k0s = smem_u32(sK + stage * C::TILE_BYTES);
+            // descriptors built once per tile; a K step moves only the start
+            // address field (bits 0..13, address / 16), which cannot carry
+            const uint64_t qd = sdesc_kmajor(q0);
+            const uint64_t kd = sdesc_kmajor(smem_u32(sK + stage * C::TILE_BYTES));
 #pragma unroll
             for (int k = 0; k < DH / 16; ++k) {
-              const uint32_t off = (k / 4) * (kTile * 128) + (k % 4) * 32;
-              mma_ss(tS(nj % 3), sdesc_kmajor(q0 + off), sdesc_kmajor(k0s + off), C::IDESC_S, k > 0);
+              const uint32_t off = ((k / 4) * (kTile * 128) + (k % 4) * 32) >> 4;
+              mma_ss(tS(nj % 3), qd + off, kd + off, C::IDESC_S, k > 0);
             }
             mma_commit(&s_full[nj % 3]);
             mma_commit(&k_empty[stage]);
@@ -470,10 +473,10 @@ __global__ void __launch_bounds__(352, 1)
             if (!mbar_wait(&v_full[pst], (np / C::V_STAGES) & 1, abort_flag, P.status)) { ok = false; break; }
             if (!mbar_wait(&p_full[np % 3], (np / 3) & 1, abort_flag, P.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t v0 = smem_u32(sV + pst * C::TILE_BYTES);
+            const uint64_t vd = sdesc_mnmajor(smem_u32(sV + pst * C::TILE_BYTES), kTile * 128);
 #pragma unroll
             for (int k = 0; k < kTile / 16; ++k)
-              mma_ts(tO, tP(np % 3) + k * 8, sdesc_mnmajor(v0 + k * 2048, kTile * 128), C::IDESC_O,
+              mma_ts(tO, tP(np % 3) + k * 8, vd + (uint64_t)(k * 2048 >> 4), C::IDESC_O,
                      (j > 2 || k > 0) ? 1u : 0u);
             mma_commit(&v_empty[pst]);
           }

@@ -50,6 +50,7 @@ from hstu_sequential_transducer_b200 import workloads as W  # noqa: E402
 
 METRIC = "HSTU layer fwd+bwd tokens/s and TFLOP/s at max_len 8192; % of B200 BF16 peak"
 FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+MUFU_TOPS = 148 * 16 * 1.965e9 / 1e12          # tanh.approx results per second, T/s
 
 
 def pairs_allowed(lengths, num_targets=None):
@@ -412,13 +413,18 @@ def run_ours(args):
         # read dZ, O (fp32), U, Pre_U, statistics; write dO and dPre_U
         "ln_bwd": ("hbm", w.T * (14 * d + 8)),
     }
-    # contractions that run on the FP32 pipes (fp32 layers; attention at
-    # dh = 32) are held against the FP32 FMA peak: 148 SMs x 128 lanes x
-    # 2 flops x 1.965 GHz = 74.4 TFLOP/s
+    # contractions that run on the FP32 pipes (fp32 layers) are held against
+    # the FP32 FMA peak: 148 SMs x 128 lanes x 2 flops x 1.965 GHz = 74.4
+    # TFLOP/s.  bf16 heads of 32 run on the tensor cores zero-padded to 64
+    # columns, where one tanh per allowed score (the MUFU unit) binds before
+    # the tensor pipe: held against 148 SMs x 16 MUFU results x 1.965 GHz
     dh = d // w.num_heads
-    if w.dtype == "f32" or dh == 32:
+    if w.dtype == "f32":
         for k in ("attn_fwd", "attn_bwd"):
             per_launch[k] = ("alu", per_launch[k][1])
+    elif dh == 32:
+        per_launch["attn_fwd"] = ("mufu", w.num_heads * pairs)
+        per_launch["attn_bwd"] = ("mufu", w.num_heads * pairs)
     if w.dtype == "f32":
         for k in ("proj_in", "proj_out", "proj_in_bwd", "proj_out_bwd"):
             per_launch[k] = ("alu", per_launch[k][1])
@@ -447,13 +453,25 @@ def run_ours(args):
                 ach = work / avg_s / 1e12
                 peak = FP32_FMA_TFLOPS
                 unit, src = "TFLOP/s", "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"
+            elif bound == "mufu":
+                ach = work / avg_s / 1e12
+                peak = MUFU_TOPS
+                unit, src = "Ttanh/s", "derived: 148 SMs x 16 MUFU results/clk x 1.965 GHz"
             else:
                 ach = work / avg_s / 1e9
                 peak = peaks.get("hbm_gbs")
                 unit, src = "GB/s", f"{peak_src} (hbm_gbs)"
-            roof = {"kernel": top, "bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+            roof = {"kernel": top, "bound": "alu" if bound == "mufu" else bound,
+                    "achieved": ach, "peak": peak, "unit": unit,
                     "frac": ach / peak, "traffic": profiled_traffic(top, w.name),
                     "peak_source": src, "work_per_launch": work}
+            if bound == "mufu":
+                # the same launch against the bf16 tensor roof (algorithmic
+                # flops 4 d per allowed pair; the padded columns not counted)
+                fl = (4 if top == "attn_fwd" else 8) * d * pairs
+                tpk = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+                roof["tensor"] = {"achieved": fl / avg_s / 1e12, "peak": tpk, "unit": "TFLOP/s",
+                                  "frac": fl / avg_s / 1e12 / tpk}
 
     # end to end through the public API with host buffers
     e2e = None

@@ -119,7 +119,8 @@ FwdWs fwd_ws(const hstu_config* c, int B, int64_t T) {
   w.z = align_up(w.o + t * d * 4, 256);
   w.xlow = align_up(w.z + t * d * es, 256);
   w.attn = align_up(w.xlow + (c->io_dtype != c->dtype ? t * d * es : 0), 256);
-  w.total = align_up(w.attn + attention_fwd_ws(B, T, c->num_heads, c->max_seq_len), 256);
+  w.total = align_up(
+      w.attn + attention_fwd_ws_full(c->dtype, B, T, c->num_heads, c->head_dim), 256);
   return w;
 }
 
@@ -136,7 +137,7 @@ BwdWs bwd_ws(const hstu_config* c, int B, int64_t T) {
   w.dq = align_up(w.dpre + t * 4 * d * es, 256);
   w.dylow = align_up(w.dq + t * d * 4, 256);
   w.attn = align_up(w.dylow + (c->io_dtype != c->dtype ? t * d * es : 0), 256);
-  w.total = align_up(w.attn + attention_bwd_ws(B, T, c->num_heads, c->d_model, c->max_seq_len), 256);
+  w.total = align_up(w.attn + attention_bwd_ws(c->dtype, B, T, c->num_heads, c->head_dim), 256);
   return w;
 }
 
@@ -480,12 +481,12 @@ hstu_status hstu_saved_layout(const hstu_config* cfg, int64_t T,
 
 size_t hstu_attention_workspace_size(const hstu_config* cfg, int32_t B, int64_t T) {
   if (check_cfg(cfg) != HSTU_OK || B < 0 || T < 0) return 0;
-  return attention_fwd_ws(B, T, cfg->num_heads, cfg->max_seq_len);
+  return attention_fwd_ws_full(cfg->dtype, B, T, cfg->num_heads, cfg->head_dim);
 }
 
 size_t hstu_attention_bwd_workspace_size(const hstu_config* cfg, int32_t B, int64_t T) {
   if (check_cfg(cfg) != HSTU_OK || B < 0 || T < 0) return 0;
-  return align_up(attention_bwd_ws(B, T, cfg->num_heads, cfg->d_model, cfg->max_seq_len), 256) +
+  return align_up(attention_bwd_ws(cfg->dtype, B, T, cfg->num_heads, cfg->head_dim), 256) +
          align_up((size_t)T * cfg->d_model * 4, 256);
 }
 
@@ -541,7 +542,7 @@ hstu_status hstu_attention_fwd(const hstu_config* cfg, const float* rab_pos, con
   HSTU_TRY(need(o_out, T));
   HSTU_TRY(meta(rab_pos, rab_pos ? 1 : 0, 4));
   HSTU_TRY(meta(rab_time, rab_time ? 1 : 0, 4));
-  const size_t need_ws = attention_fwd_ws(B, T, cfg->num_heads, cfg->max_seq_len);
+  const size_t need_ws = attention_fwd_ws(B, T, cfg->num_heads);
   if (ws_bytes < need_ws) return HSTU_ERR_WORKSPACE;
   if (need_ws > 0) HSTU_TRY(need(workspace, 1));
   if (T == 0 || B == 0) return HSTU_OK;
@@ -562,7 +563,7 @@ hstu_status hstu_softmax_attention_fwd(const hstu_config* cfg, const float* rab_
   HSTU_TRY(need(o_out, T));
   HSTU_TRY(meta(rab_pos, rab_pos ? 1 : 0, 4));
   HSTU_TRY(meta(rab_time, rab_time ? 1 : 0, 4));
-  const size_t need_ws = attention_fwd_ws(B, T, cfg->num_heads, cfg->max_seq_len);
+  const size_t need_ws = attention_fwd_ws(B, T, cfg->num_heads);
   if (ws_bytes < need_ws) return HSTU_ERR_WORKSPACE;
   if (need_ws > 0) HSTU_TRY(need(workspace, 1));
   if (T == 0 || B == 0) return HSTU_OK;
@@ -590,7 +591,7 @@ hstu_status hstu_attention_fwd_cached(const hstu_config* cfg, const float* rab_p
   HSTU_TRY(need(o_out, Tc));
   HSTU_TRY(meta(rab_pos, rab_pos ? 1 : 0, 4));
   HSTU_TRY(meta(rab_time, rab_time ? 1 : 0, 4));
-  const size_t need_ws = attention_fwd_ws(B, Tc, cfg->num_heads, cfg->max_seq_len);
+  const size_t need_ws = attention_fwd_ws(B, Tc, cfg->num_heads);
   if (ws_bytes < need_ws) return HSTU_ERR_WORKSPACE;
   if (need_ws > 0) HSTU_TRY(need(workspace, 1));
   if (Tc == 0 || B == 0) return HSTU_OK;
@@ -691,8 +692,8 @@ hstu_status hstu_attention_bwd(const hstu_config* cfg, const float* rab_pos,
   HSTU_TRY(meta(rab_time, rab_time ? 1 : 0, 4));
   HSTU_TRY(meta(drab_pos, drab_pos ? 1 : 0, 4));
   HSTU_TRY(meta(drab_time, drab_time ? 1 : 0, 4));
-  const size_t attn = align_up(attention_bwd_ws(B, T, cfg->num_heads, cfg->d_model,
-                                                cfg->max_seq_len), 256);
+  const size_t attn = align_up(attention_bwd_ws(cfg->dtype, B, T, cfg->num_heads,
+                                                cfg->head_dim), 256);
   if (ws_bytes < hstu_attention_bwd_workspace_size(cfg, B, T)) return HSTU_ERR_WORKSPACE;
   if (T == 0 || B == 0) return HSTU_OK;
   HSTU_TRY(need(workspace, 1));

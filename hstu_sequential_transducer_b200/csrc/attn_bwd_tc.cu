@@ -36,6 +36,7 @@
 
 #include <type_traits>
 
+#include "attn_sched.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -48,6 +49,7 @@ namespace {
 
 constexpr int kT = 128;
 constexpr int kMaxCostB = 514;
+static_assert(kMaxCostB <= kScanThreads, "one scan thread per cost bin");
 
 struct BItem {
   int32_t b;
@@ -91,13 +93,7 @@ __global__ void bsched_count(AttnArgs a, BSched w) {
   }
 }
 __global__ void bsched_scan(BSched w) {
-  if (threadIdx.x != 0) return;
-  int run = 0;
-  for (int c = kMaxCostB - 1; c >= 0; --c) {
-    w.cursor[c] = run;
-    run += w.hist[c];
-  }
-  *w.total = run;
+  scan_descending(w.hist, w.cursor, w.total, kMaxCostB);
 }
 __global__ void bsched_fill(AttnArgs a, BSched w) {
   for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < a.B; b += gridDim.x * blockDim.x) {
@@ -453,6 +449,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     constexpr uint32_t kAct = 32 * kActWarps;
     const int d = P.A.d;
+    const int odh = a.o_dh > 0 ? a.o_dh : DH;        // dQ, dPre columns stored per head
     uint32_t items_done = 0, m = 0;
     int cur_h = -1;
     const float inv_N = a.inv_N;
@@ -614,10 +611,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
         if (named_barrier_any(1, kAct, fail)) { fail = true; break; }
         tc_fence_after();
         const int qrow = q0 + row;
-        float* dq = P.A.dq_acc + (s0 + qrow) * (int64_t)d + item.h * DH;
+        float* dq = P.A.dq_acc + (s0 + qrow) * (int64_t)d + item.h * odh;
 #pragma unroll 1
         for (int cc = 0; cc < DH / 64; ++cc) {
           const int c = wg * (DH / 64) + cc;
+          if (c * 32 >= odh) continue;                 // zero-padded head columns
           uint32_t r[32];
           tmem_ld32(tA + lane_off + c * 32, r);
           tmem_ld_wait();
@@ -644,12 +642,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll 1
       for (int cc = 0; cc < DH / 64; ++cc) {
         const int c = wg * (DH / 64) + cc;
+        if (c * 32 >= odh) continue;                   // zero-padded head columns
         uint32_t rv[32], rk[32];
         tmem_ld32(tdV + lane_off + c * 32, rv);
         tmem_ld32(tdK + lane_off + c * 32, rk);
         tmem_ld_wait();
         if (kvalid) {
-          const int col = item.h * DH + c * 32;
+          const int col = item.h * odh + c * 32;
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
             const uint4 pv4 = *reinterpret_cast<const uint4*>(pre + rowoff + d + col + i);
@@ -1402,7 +1401,7 @@ cudaError_t launch_bwd(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaStr
   if (e != cudaSuccess) return e;
   const int blocks = (a.B + 255) / 256;
   bsched_count<<<blocks, 256, 0, s>>>(a, w);
-  bsched_scan<<<1, 32, 0, s>>>(w);
+  bsched_scan<<<1, kScanThreads, 0, s>>>(w);
   bsched_fill<<<blocks, 256, 0, s>>>(a, w);
   count_launch(3);
   BParams P;
@@ -1435,7 +1434,7 @@ cudaError_t launch_bwd3(const AttnBwdArgs& A, void* ws, uint32_t* status, cudaSt
   if (e != cudaSuccess) return e;
   const int blocks = (a.B + 255) / 256;
   bsched_count<<<blocks, 256, 0, s>>>(a, w);
-  bsched_scan<<<1, 32, 0, s>>>(w);
+  bsched_scan<<<1, kScanThreads, 0, s>>>(w);
   bsched_fill<<<blocks, 256, 0, s>>>(a, w);
   count_launch(3);
   BParams P;

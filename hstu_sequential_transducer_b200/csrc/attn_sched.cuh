@@ -27,6 +27,41 @@ struct SchedWs {
   AttnItem* items;   // [max_items]
 };
 
+// Threads of the one-block scan kernels of the counting sorts: at least one
+// per cost bin, whole warps.
+constexpr int kScanThreads = (kMaxCost + 31) / 32 * 32;
+
+// Exclusive scan of hist[0, n) in descending bin order, by one block of
+// blockDim.x >= n threads (whole warps, at most 1024): cursor[c] = sum of
+// hist[c'] over c' > c, and *total = the sum of all bins.
+__device__ __forceinline__ void scan_descending(const int32_t* hist, int32_t* cursor,
+                                                int32_t* total, int n) {
+  __shared__ int32_t warp_sum[32];
+  const int t = threadIdx.x, lane = t & 31, wid = t >> 5, nw = blockDim.x >> 5;
+  const int c = n - 1 - t;                       // thread t holds the t-th largest bin
+  const int v = c >= 0 ? hist[c] : 0;
+  int x = v;                                     // inclusive scan within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sum[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int sw = lane < nw ? warp_sum[lane] : 0;     // inclusive scan of the warp sums
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, sw, o);
+      if (lane >= o) sw += y;
+    }
+    if (lane < nw) warp_sum[lane] = sw;
+  }
+  __syncthreads();
+  if (c >= 0) cursor[c] = (wid > 0 ? warp_sum[wid - 1] : 0) + x - v;
+  if (t == 0) *total = warp_sum[nw - 1];
+}
+
 SchedWs sched_ws(void* ws);
 // Fills the work list in `ws` (attn_sched_bytes of it) on stream s.
 cudaError_t build_schedule(const AttnArgs& a, void* ws, cudaStream_t s);

@@ -76,15 +76,9 @@ __global__ void sched_count_kernel(AttnArgs a, SchedWs w) {
   }
 }
 
-// One warp: cursor[c] = number of items of cost > c (descending order).
+// cursor[c] = number of items of cost > c (descending order).
 __global__ void sched_scan_kernel(SchedWs w) {
-  if (threadIdx.x != 0) return;
-  int run = 0;
-  for (int c = kMaxCost - 1; c >= 0; --c) {
-    w.cursor[c] = run;
-    run += w.hist[c];
-  }
-  *w.total = run;
+  scan_descending(w.hist, w.cursor, w.total, kMaxCost);
 }
 
 __global__ void sched_fill_kernel(AttnArgs a, SchedWs w) {
@@ -111,7 +105,7 @@ cudaError_t build_schedule(const AttnArgs& a, void* ws, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int blocks = (a.B + 255) / 256;
   sched_count_kernel<<<blocks, 256, 0, s>>>(a, w);
-  sched_scan_kernel<<<1, 32, 0, s>>>(w);
+  sched_scan_kernel<<<1, kScanThreads, 0, s>>>(w);
   sched_fill_kernel<<<blocks, 256, 0, s>>>(a, w);
   count_launch(3);
   return cudaGetLastError();
@@ -638,9 +632,11 @@ __global__ void __launch_bounds__(352, 1)
         tc_fence_after();
       }
       const bf16* sv = static_cast<const bf16*>(a.self_v) + (g.qs + r0 + row) * a.q_stride + h * DH;
+      const int odh = a.o_dh > 0 ? a.o_dh : DH;       // O columns stored per head
 #pragma unroll
       for (int cc = 0; cc < DH / 64; ++cc) {
         const int c = wg * (DH / 64) + cc;            // 32-column chunk of O
+        if (c * 32 >= odh) continue;                   // zero-padded head columns
         float o[32];
         if (nk > 0) {
           uint32_t r[32];
@@ -666,7 +662,7 @@ __global__ void __launch_bounds__(352, 1)
               }
             }
           }
-          float* dst = O + (g.qs + r0 + row) * a.o_stride + h * DH + c * 32;
+          float* dst = O + (g.qs + r0 + row) * a.o_stride + h * odh + c * 32;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4*>(dst + i) =

@@ -73,6 +73,9 @@ struct AttnArgs {
   const float* rab_pos = nullptr;
   const float* rab_time = nullptr;
   float inv_N = 1.0f;
+  // Columns of O per head when they differ from dh: heads of 32 zero-padded
+  // to 64 run with dh = 64 and store only their first o_dh columns.
+  int o_dh = 0;
 };
 
 struct AttnBwdArgs {
@@ -90,11 +93,18 @@ struct AttnBwdArgs {
 cudaError_t attention_fwd(int dtype, const AttnArgs& a, void* ws, size_t ws_bytes, cudaStream_t s);
 cudaError_t attention_bwd(int dtype, const AttnBwdArgs& a, void* ws, size_t ws_bytes,
                           cudaStream_t s);
-size_t attention_fwd_ws(int B, int64_t T, int H, int max_len);
+// Workspace of the attention forward: the work list (required) and, for bf16
+// head_dim 32, a zero-padded copy of V|Q|K (optional: with it those heads run
+// on the tensor-core kernel, without it on the CUDA-core one).
+size_t attention_fwd_ws(int B, int64_t T, int H);
+size_t attention_fwd_pad_bytes(int dtype, int64_t T, int H, int dh);
+size_t attention_fwd_ws_full(int dtype, int B, int64_t T, int H, int dh);
 size_t attn_sched_bytes(int B, int64_t Tq, int H);
 bool attention_fwd_tc_supported(int dtype, const AttnArgs& a);
 cudaError_t attention_fwd_tc(const AttnArgs& a, void* ws, uint32_t* status, cudaStream_t s);
-size_t attention_bwd_ws(int B, int64_t T, int H, int d, int max_len);
+// Backward workspace: the work list and, for bf16 head_dim 32, zero-padded
+// copies of V|Q|K and dO (the head_dim-64 tensor-core kernel runs on them).
+size_t attention_bwd_ws(int dtype, int B, int64_t T, int H, int dh);
 size_t attn_bwd_sched_bytes(int B, int64_t T, int H);
 bool attention_bwd_tc_supported(int dtype, const AttnBwdArgs& a);
 cudaError_t attention_bwd_tc(const AttnBwdArgs& a, void* ws, uint32_t* status, cudaStream_t s);
@@ -123,6 +133,11 @@ cudaError_t dq_finalize(int dtype, const float* dq_acc, const void* pre_q, int64
                         void* dpre_q, int64_t T, int d, cudaStream_t s);
 cudaError_t copy_columns(int dtype, const void* src, int64_t src_stride, void* dst,
                          int64_t dst_stride, int64_t rows, int64_t cols, cudaStream_t s);
+// dst [T][nblk*H*64] = blocks b0 (, b1, b2) of every token, bf16, each head's
+// 32 values followed by 32 zeros; source rows ss elements apart, 16-byte
+// aligned; nblk in 1..3.
+cudaError_t pad_heads32(const void* b0, const void* b1, const void* b2, int nblk, int64_t ss,
+                        void* dst, int64_t T, int H, cudaStream_t s);
 cudaError_t convert_f32_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t s);
 cudaError_t validate_inputs(const int64_t* offs, int B, int64_t T, const int64_t* ts,
                             const int32_t* nt, int max_len, uint32_t* flags, cudaStream_t s);

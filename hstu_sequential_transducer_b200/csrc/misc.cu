@@ -78,6 +78,27 @@ __global__ void copy_columns_kernel(const T* __restrict__ src, int64_t ss, T* __
   }
 }
 
+// One 16-byte chunk of the padded copy per thread: chunks 0-3 of a head hold
+// its 32 values, chunks 4-7 zeros.
+__global__ void pad_heads32_kernel(const bf16* __restrict__ b0, const bf16* __restrict__ b1,
+                                   const bf16* __restrict__ b2, int nblk, int64_t ss,
+                                   uint4* __restrict__ dst, int64_t T, int H) {
+  const int64_t per_row = (int64_t)nblk * H * 8;
+  const int64_t n = T * per_row;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / per_row;
+    const int rem = (int)(i - r * per_row);
+    const int blk = rem / (H * 8), h = (rem / 8) % H, j = rem % 8;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (j < 4) {
+      const bf16* src = blk == 0 ? b0 : (blk == 1 ? b1 : b2);
+      val = *reinterpret_cast<const uint4*>(src + r * ss + h * 32 + j * 8);
+    }
+    dst[i] = val;
+  }
+}
+
 __global__ void convert_kernel(const float* __restrict__ src, bf16* __restrict__ dst, int64_t n) {
   const int64_t n8 = n / 8;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
@@ -178,6 +199,17 @@ cudaError_t copy_columns(int dtype, const void* src, int64_t ss, void* dst, int6
     copy_columns_kernel<bf16><<<g, 256, 0, s>>>((const bf16*)src, ss, (bf16*)dst, ds, rows, cols);
   else
     copy_columns_kernel<float><<<g, 256, 0, s>>>((const float*)src, ss, (float*)dst, ds, rows, cols);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t pad_heads32(const void* b0, const void* b1, const void* b2, int nblk, int64_t ss,
+                        void* dst, int64_t T, int H, cudaStream_t s) {
+  if (T == 0 || H == 0) return cudaSuccess;
+  if (nblk < 1 || nblk > 3) return cudaErrorInvalidValue;
+  const unsigned g = grid_for(T * nblk * H * 8, 256);
+  pad_heads32_kernel<<<g, 256, 0, s>>>((const bf16*)b0, (const bf16*)b1, (const bf16*)b2, nblk,
+                                       ss, (uint4*)dst, T, H);
   count_launch();
   return cudaGetLastError();
 }

@@ -66,7 +66,9 @@ extern "C" hstu_status hstu_attention_fwd_noalloc(const hstu_config* cfg, const 
                                             timestamps, num_targets, o_out, nullptr, 0, stream);
   if (st != HSTU_ERR_WORKSPACE) return st;
   if (B == 0 || T == 0) return HSTU_OK;  // nothing to compute; the scratch is not touched
-  const size_t need = hstu_attention_workspace_size(cfg, B, T);
+  // The work list must fit; bf16 heads of 32 also use the scratch left after
+  // it for their zero-padded copy when that fits too (else the CUDA-core kernel).
+  const size_t need = hstu::attention_fwd_ws(B, T, cfg->num_heads);
   if (need > kNoAllocScratchBytes) return HSTU_ERR_WORKSPACE;  // beyond the static scratch
   int err = 0;
   void* ws = noalloc_scratch(&err);

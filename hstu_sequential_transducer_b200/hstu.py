@@ -198,6 +198,10 @@ def workspace_size(cfg: Config, B: int, T: int):
     return ws.value, sv.value
 
 
+def attention_workspace_size(cfg: Config, B: int, T: int) -> int:
+    return int(lib().hstu_attention_workspace_size(ctypes.byref(cfg), B, T))
+
+
 def saved_layout(cfg: Config, T: int):
     off = (c_size_t * (SAVED_COUNT + 1))()
     _check(lib().hstu_saved_layout(ctypes.byref(cfg), T, off), "hstu_saved_layout")
@@ -247,13 +251,17 @@ def proj_in_fwd(cfg, w: LayerWeights, x, pre_out, g_out, stream=None):
                                   ptr(pre_out), ptr(g_out), stream_ptr(stream)), "hstu_proj_in_fwd")
 
 
-def attention_fwd(cfg, rab_pos, rab_time, g, offsets, timestamps, num_targets, o_out, stream=None):
+def attention_fwd(cfg, rab_pos, rab_time, g, offsets, timestamps, num_targets, o_out, stream=None,
+                  ws_bytes=None):
+    """ws_bytes: workspace bytes passed to the call (default: the full
+    hstu_attention_workspace_size)."""
     B, T = offsets.numel() - 1, g.shape[0]
     n = lib().hstu_attention_workspace_size(ctypes.byref(cfg), B, T)
     ws = workspace(n, g.device, "attn")
+    nb = ws.numel() if ws_bytes is None else min(int(ws_bytes), ws.numel())
     _check(lib().hstu_attention_fwd(ctypes.byref(cfg), ptr(rab_pos), ptr(rab_time), ptr(g),
                                     ptr(offsets), B, T, ptr(timestamps), ptr(num_targets),
-                                    ptr(o_out), ptr(ws), ws.numel(), stream_ptr(stream)),
+                                    ptr(o_out), ptr(ws), nb, stream_ptr(stream)),
            "hstu_attention_fwd")
 
 

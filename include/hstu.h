@@ -164,9 +164,10 @@ hstu_status hstu_proj_in_fwd(const hstu_config* cfg, const hstu_weights* w,
                              cudaStream_t stream);
 
 /* Equation (2) for every head, with rab^{p,t} bucketing, the causal or
- * M-FALCON mask, and ragged work partitioning (no padding is computed).
+ * M-FALCON mask, and ragged work partitioning (sequences are not padded).
  * g [T][4d] holds U|V|Q|K of every token; o_out [T][d] fp32.
- * workspace: at least hstu_attention_workspace_size(B, T) bytes. */
+ * workspace: hstu_attention_workspace_size(B, T) bytes; less than its
+ * work-list part returns HSTU_ERR_WORKSPACE. */
 hstu_status hstu_attention_fwd(const hstu_config* cfg, const float* rab_pos,
                                const float* rab_time, const void* g,
                                const int64_t* seq_offsets, int32_t B, int64_t T,
@@ -191,8 +192,10 @@ hstu_status hstu_attention_fwd_cached(const hstu_config* cfg, const float* rab_p
 /* hstu_attention_fwd for callers that cannot allocate device memory (the
  * paper has no counterpart: this is a property of this library's interface).
  * Same arguments and result as hstu_attention_fwd, without the workspace: the
- * scratch (the work list of the tensor-core kernel) lives in a 2 MiB static
- * device array that every GPU loading the library keeps until process exit.
+ * scratch (the work list of the tensor-core kernel, and for bf16 head_dim 32
+ * the zero-padded copy of V|Q|K when it fits after it) lives in a 2 MiB
+ * static device array that every GPU loading the library keeps until process
+ * exit.
  * Meant for processes held to a device-memory budget fixed at start-up, which
  * may not allocate while serving, and for C hosts that own only their input
  * and output buffers.
@@ -230,7 +233,15 @@ hstu_status hstu_softmax_attention_fwd(const hstu_config* cfg, const float* rab_
                                        void* o_out, void* workspace, size_t ws_bytes,
                                        cudaStream_t stream);
 
-/* Bytes of workspace the attention entry points need. Host only. */
+/* Bytes of workspace the attention entry points need. Host only.
+ * The work list of the tensor-core kernel is required.  For bf16 with
+ * head_dim 32 the size also holds a copy of V|Q|K with every head
+ * zero-padded to 64 columns (T * 3 * H * 64 * 2 bytes, after the work list
+ * rounded up to 256 bytes): with it those heads run on the head_dim-64
+ * tensor-core kernel; hstu_attention_fwd given a workspace that holds the
+ * work list but not the copy runs them on the CUDA-core kernel instead.
+ * hstu_attention_fwd_cached and hstu_softmax_attention_fwd never use the
+ * copy. */
 size_t hstu_attention_workspace_size(const hstu_config* cfg, int32_t B, int64_t T);
 
 /* Equation (3), first half: Z = (LayerNorm(O) * gamma + beta) (.) U.

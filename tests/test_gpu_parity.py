@@ -192,6 +192,40 @@ def test_attention_fwd_parity(dtype, dh, targets):
     check_el(np_(o), ref, dtype, "O")
 
 
+def test_attention_fwd_head32_paths():
+    """bf16 heads of 32 columns.  With the full workspace they are copied
+    zero-padded to 64 columns and run on the head_dim-64 tensor-core kernel
+    (launches: the work list's three, the padding copy, the attention kernel);
+    with a workspace that holds the work list only, they run on the CUDA-core
+    kernel (one launch).  Both match the oracle, tiles, ragged tails and
+    M-FALCON candidates included."""
+    Hh, dh = 4, 32
+    d = Hh * dh
+    lengths = [700, 1, 0, 129, 64, 65, 257, 1000]
+    nt = [40, 1, 0, 129, 0, 7, 100, 300]
+    w = W.custom(lengths, d=d, H=Hh, dtype="bf16", N=700.0, num_targets=nt, mean_gap=3000.0,
+                 seed=32)
+    rng = np.random.default_rng(320)
+    g = rand_g(rng, w.T, d, "bf16", scale=0.5)
+    dw = S.DeviceWorkload.from_workload(w)
+    gd = dev_rows(g, "bf16")
+    p = w.params[0]
+    ref = R.attention_forward(g, w.seq_offsets, w.timestamps, w.num_targets, p.rab_pos,
+                              p.rab_time, lcfg(w))
+    full = H.attention_workspace_size(dw.cfg, w.B, w.T)
+    pad = w.T * 3 * Hh * 64 * 2
+    for ws_bytes, launches in ((full, 5), (full - pad, 1)):
+        o = nan_out(w.T, d)
+        torch.cuda.synchronize()
+        n0 = H.launch_count()
+        H.attention_fwd(dw.cfg, dw.layers[0].rab_pos, dw.layers[0].rab_time, gd, dw.offsets,
+                        dw.timestamps, dw.num_targets, o, ws_bytes=ws_bytes)
+        torch.cuda.synchronize()
+        assert H.launch_count() - n0 == launches
+        assert H.device_status() == 0
+        check_el(np_(o), ref, "bf16", f"O (workspace {ws_bytes} bytes)")
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("d", [64, 512, 1024])
 def test_ln_gate_fwd_parity(dtype, d):
@@ -309,8 +343,16 @@ def test_attention_bwd_parity(dtype, dh, targets):
     dpre = nan_out(w.T, 4 * d, dtype=cdt(dtype))     # the V, Q and K blocks are written
     drp = torch.zeros_like(lw.rab_pos)
     drt = torch.zeros_like(lw.rab_time)
+    torch.cuda.synchronize()
+    n0 = H.launch_count()
     H.attention_bwd(dw.cfg, lw.rab_pos, lw.rab_time, dev_rows(g, dtype), dev_rows(pre, dtype),
                     dev_rows(dout, dtype), dw.offsets, dw.timestamps, dw.num_targets, dpre, drp, drt)
+    torch.cuda.synchronize()
+    if dtype == "bf16" and dh == 32:
+        # heads of 32 on the head_dim-64 tensor-core kernel: two padding
+        # copies, the work list's three launches, the kernel, the candidates'
+        # self term (with targets) and the dQ fold-in
+        assert H.launch_count() - n0 == (8 if targets else 7)
     p = w.params[0]
     dg, rdp, rdt = R.attention_backward(g, dout, w.seq_offsets, w.timestamps, w.num_targets,
                                         p.rab_pos, p.rab_time, lcfg(w))

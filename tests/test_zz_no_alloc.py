@@ -60,11 +60,13 @@ def _noalloc(cfg, rp, rt, g, offs, ts, nt, out, B=None, T=None):
                                               H.stream_ptr())
 
 
-@pytest.mark.parametrize("dtype,dh", [("bf16", 128), ("f32", 32)])
+@pytest.mark.parametrize("dtype,dh", [("bf16", 128), ("bf16", 32), ("f32", 32)])
 def test_noalloc_matches_attention_fwd_twice(dtype, dh):
     """Two calls in a row (different inputs: the second must not see the first
     one's work list) equal hstu_attention_fwd bit for bit; bf16 dh 128 runs the
-    tensor-core kernel, fp32 dh 32 the CUDA-core one."""
+    tensor-core kernel, bf16 dh 32 the same kernel on heads zero-padded to 64
+    columns (the padded copy also fits in the scratch), fp32 dh 32 the
+    CUDA-core one."""
     for i, seed in enumerate((21, 22)):
         cfg, rp, rt, g, offs, ts, nt, T, d = _inputs(seed, dtype, dh)
         ref = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")

@@ -78,24 +78,27 @@ __global__ void copy_columns_kernel(const T* __restrict__ src, int64_t ss, T* __
   }
 }
 
-// One 16-byte chunk of the padded copy per thread: chunks 0-3 of a head hold
-// its 32 values, chunks 4-7 zeros.
+// One warp per token row, one 16-byte chunk per lane and pass: chunks 0-3 of
+// a head hold its 32 values, chunks 4-7 zeros.
 __global__ void pad_heads32_kernel(const bf16* __restrict__ b0, const bf16* __restrict__ b1,
                                    const bf16* __restrict__ b2, int nblk, int64_t ss,
                                    uint4* __restrict__ dst, int64_t T, int H) {
-  const int64_t per_row = (int64_t)nblk * H * 8;
-  const int64_t n = T * per_row;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = i / per_row;
-    const int rem = (int)(i - r * per_row);
-    const int blk = rem / (H * 8), h = (rem / 8) % H, j = rem % 8;
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (j < 4) {
-      const bf16* src = blk == 0 ? b0 : (blk == 1 ? b1 : b2);
-      val = *reinterpret_cast<const uint4*>(src + r * ss + h * 32 + j * 8);
+  const int per_row = nblk * H * 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < T;
+       r += nwarps) {
+    uint4* drow = dst + r * per_row;
+    for (int c = lane; c < per_row; c += 32) {
+      const int q = c >> 3, j = c & 7;
+      const int blk = q / H, h = q - blk * H;
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (j < 4) {
+        const bf16* src = blk == 0 ? b0 : (blk == 1 ? b1 : b2);
+        val = *reinterpret_cast<const uint4*>(src + r * ss + h * 32 + j * 8);
+      }
+      drow[c] = val;
     }
-    dst[i] = val;
   }
 }
 
@@ -207,7 +210,7 @@ cudaError_t pad_heads32(const void* b0, const void* b1, const void* b2, int nblk
                         void* dst, int64_t T, int H, cudaStream_t s) {
   if (T == 0 || H == 0) return cudaSuccess;
   if (nblk < 1 || nblk > 3) return cudaErrorInvalidValue;
-  const unsigned g = grid_for(T * nblk * H * 8, 256);
+  const unsigned g = grid_for(T, 8);            // eight rows (warps) per block
   pad_heads32_kernel<<<g, 256, 0, s>>>((const bf16*)b0, (const bf16*)b1, (const bf16*)b2, nblk,
                                        ss, (uint4*)dst, T, H);
   count_launch();

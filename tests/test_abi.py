@@ -154,3 +154,23 @@ def test_saved_activation_budget_within_14d(L, d, nh):
     per_token = off[-1] / T
     assert per_token <= 24 * d + 8 + 1e-3 * d
     assert per_token <= 2 * 14 * d
+
+
+def test_attention_workspace_holds_the_padded_head32_copy(L):
+    """bf16 heads of 32 get a zero-padded copy of V|Q|K (forward) and of
+    V|Q|K and dO (backward) in the attention workspace, after the work list
+    rounded up to 256 bytes; fp32 heads of 32 and heads of 64 get none."""
+    B, T, nh = 7, 1000, 2
+    al = lambda v: (v + 255) // 256 * 256
+    f = lambda c: L.hstu_attention_workspace_size(ctypes.byref(c), B, T)
+    b = lambda c: L.hstu_attention_bwd_workspace_size(ctypes.byref(c), B, T)
+    c32, c64 = cfg(d=64, H=nh), cfg(d=128, H=nh)
+    c32f = cfg(d=64, H=nh, dtype=H.HSTU_F32)
+    assert c32.head_dim == 32 and c64.head_dim == 64
+    sched = f(c64)                                   # the work list alone (same B, T, H)
+    assert f(c32f) == sched
+    assert f(c32) == al(sched) + T * 3 * nh * 64 * 2
+    # backward: work list (+ padding) rounded to 256, then the fp32 dQ [T][d]
+    dq32 = al(T * 64 * 4)
+    assert b(c32f) < b(c32)
+    assert b(c32) - dq32 >= T * 4 * nh * 64 * 2

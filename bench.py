@@ -23,7 +23,9 @@ dh=128), measured on rank 0 after the timed steps.
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on this host's cores (rank 0 only).
 
---attention-8k prints only that attention measurement, on its own line.
+--attention-8k prints only that attention measurement, on its own line;
+--softmax-8k the same measurement with the softmax comparison kernel's
+forward as the value (the pointwise forward beside it).
 
 --sampler measures the Stochastic Length sampler instead (selection plus the
 gathers of the fp32 rows and timestamps of the training batch, alpha 1.6 by
@@ -794,6 +796,8 @@ def run_sampler(args):
 
 ATTN8K_METRIC = ("HSTU attention fwd+bwd TFLOP/s at length 8192 (16 x 8192 tokens, H=8, dh=128, "
                  "causal, pos+time rab, bf16)")
+SOFTMAX8K_METRIC = ("softmax attention fwd TFLOP/s at length 8192 (16 x 8192 tokens, H=8, dh=128, "
+                    "causal, pos+time rab, bf16; the comparison kernel)")
 
 
 def attn8k_oracle(seconds: float):
@@ -820,7 +824,32 @@ def attn8k_oracle(seconds: float):
     return flops / t_used / 1e12, f"{reps} x one 1,024-token sequence, fwd+bwd, d=1024, H=8"
 
 
-def run_attention8k(args):
+def softmax8k_oracle(seconds: float):
+    """The softmax oracle's forward on one 1,024-token sequence (d = 1,024,
+    H = 8) for about `seconds`; returns (algorithmic TFLOP/s, sample)."""
+    from oracle import hstu_ref as R
+    from oracle import softmax_ref as SR
+    rng = np.random.default_rng(43)
+    n, d, H = 1024, 1024, 8
+    offs = np.array([0, n], np.int64)
+    ts = W.draw_timestamps(rng, [n])
+    g = rng.standard_normal((n, 4 * d)) * 0.5
+    rp, rt = rng.normal(0, 0.1, (H, 32)), rng.normal(0, 0.1, (H, 32))
+    cfg = R.LayerConfig(H, 8192.0, 32, 32, 1e-5)
+    t_used, reps = 0.0, 0
+    while t_used < seconds or reps == 0:
+        t0 = time.perf_counter()
+        SR.softmax_attention_forward(g, offs, ts, None, rp, rt, cfg)
+        t_used += time.perf_counter() - t0
+        reps += 1
+    flops = 4 * d * (n * (n + 1) // 2) * reps
+    return flops / t_used / 1e12, f"{reps} x one 1,024-token sequence, softmax fwd, d=1024, H=8"
+
+
+def run_attention8k(args, softmax=False):
+    """--attention-8k (the pointwise kernels; value = fwd+bwd TFLOP/s) or
+    --softmax-8k (value = the softmax comparison kernel's forward TFLOP/s,
+    the pointwise forward beside it)."""
     import torch
 
     from hstu_sequential_transducer_b200 import build
@@ -830,9 +859,10 @@ def run_attention8k(args):
     if args.impl == "reference":
         if rank != 0:
             return 0
-        v, desc = attn8k_oracle(args.cpu_budget)
+        v, desc = (softmax8k_oracle if softmax else attn8k_oracle)(args.cpu_budget)
         print(json.dumps({
-            "metric": ATTN8K_METRIC, "value": v, "unit": "TFLOP/s", "impl": "reference",
+            "metric": SOFTMAX8K_METRIC if softmax else ATTN8K_METRIC, "value": v, "unit": "TFLOP/s",
+            "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -858,8 +888,11 @@ def run_attention8k(args):
     clk = clocks.stop()
     peaks, peak_src = read_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    line = {"metric": ATTN8K_METRIC, "value": m["tflops"], "unit": "TFLOP/s",
-            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms"],
+    sm = m["softmax_fwd"]
+    line = {"metric": SOFTMAX8K_METRIC if softmax else ATTN8K_METRIC,
+            "value": sm["tflops"] if softmax else m["tflops"], "unit": "TFLOP/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sm["ms"] if softmax else m["ms"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": m["workload"], "tokens_per_step": m["tokens"],
@@ -871,8 +904,13 @@ def run_attention8k(args):
                          "traffic": None, "peak_source": f"{peak_src} (bf16_tflops_sustained)",
                          "work_per_launch": m["attn_bwd"]["flops"]},
             "gpu_launches": launches, "clocks": clk, "e2e": None}
+    if softmax:
+        line["roofline"] = {"kernel": "softmax_fwd", "bound": "tensor", "achieved": sm["tflops"],
+                            "peak": peak, "unit": "TFLOP/s", "frac": sm["frac"], "traffic": None,
+                            "peak_source": f"{peak_src} (bf16_tflops_sustained)",
+                            "work_per_launch": sm["flops"]}
     if not args.skip_cpu:
-        v, desc = attn8k_oracle(args.cpu_budget)
+        v, desc = (softmax8k_oracle if softmax else attn8k_oracle)(args.cpu_budget)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": os.cpu_count(),
                                 "kind": "oracle", "sample": desc}
     print(json.dumps(line), flush=True)
@@ -975,13 +1013,15 @@ def main(argv=None):
     ap.add_argument("--alpha", type=float, default=1.6)
     ap.add_argument("--attention-8k", action="store_true",
                     help="measure the attention kernels alone on 16 sequences of 8,192 tokens")
+    ap.add_argument("--softmax-8k", action="store_true",
+                    help="the softmax comparison kernel alone on 16 sequences of 8,192 tokens")
     ap.add_argument("--skip-attention-8k", action="store_true",
                     help="leave the attention_8k measurement out of the default line")
     ap.add_argument("--split", action="store_true",
                     help="shard one training batch across the ranks (LPT by n^2; strong scaling)")
     args = ap.parse_args(argv)
-    if args.attention_8k:
-        return run_attention8k(args)
+    if args.attention_8k or args.softmax_8k:
+        return run_attention8k(args, softmax=args.softmax_8k)
     if args.sampler:
         return run_sampler(args)
     if args.impl == "reference":

@@ -57,6 +57,12 @@ def test_attention_8k_reference_line():
     assert d["value"] > 0
 
 
+def test_softmax_8k_reference_line():
+    d = run_line(["--softmax-8k", "--impl", "reference", "--cpu-budget", "0.1"])
+    assert KEYS <= set(d) and d["impl"] == "reference" and d["unit"] == "TFLOP/s"
+    assert d["value"] > 0 and "softmax" in d["metric"]
+
+
 def test_split_shards_partition_one_batch():
     """--split: every rank draws the same batch and keeps its LPT share; the
     shares partition the batch's sequences and tokens."""

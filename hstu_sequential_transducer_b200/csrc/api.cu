@@ -213,8 +213,11 @@ hstu_status do_ln_fwd(const hstu_config* c, const void* gamma, const void* beta,
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
+// y_low (bf16, optional): the copy of the fp32 output y that the next layer's
+// projection reads, written by the same epilogue (fp32 residual stream only).
 hstu_status do_proj_out(const hstu_config* c, const void* W2, const void* b2, const void* z,
-                        const void* x, int64_t T, void* y, cudaStream_t s) {
+                        const void* x, int64_t T, void* y, cudaStream_t s,
+                        void* y_low = nullptr) {
   const int d = c->d_model;
   GemmArgs a;
   a.A = z; a.lda = d; a.a_kmajor = true;
@@ -222,6 +225,7 @@ hstu_status do_proj_out(const hstu_config* c, const void* W2, const void* b2, co
   a.M = T; a.N = d; a.K = d;
   a.epi = x ? EPI_RESID : EPI_STORE; a.C = y; a.ldc = d; a.bias = b2; a.R = x; a.ldr = d;
   a.io_f32 = c->io_dtype == HSTU_F32;
+  if (x && a.io_f32 && c->dtype == HSTU_BF16) a.C2 = y_low;
   prof_begin(HSTU_K_PROJ_OUT, s);
   cudaError_t e = gemm(c->dtype, a, s);
   prof_end(HSTU_K_PROJ_OUT, s);
@@ -294,9 +298,11 @@ hstu_status do_attention_bwd(const hstu_config* c, const float* rp, const float*
   return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
+// dx_low (bf16, optional): the copy of the fp32 dx that the layer below's
+// backward reads as its dY operand, written by the same epilogue.
 hstu_status do_proj_in_bwd(const hstu_config* c, const void* W1, const void* x, const void* dpre,
                            const void* dy, int64_t T, void* dx, float* dW1, float* db1,
-                           cudaStream_t s) {
+                           cudaStream_t s, void* dx_low = nullptr) {
   const int d = c->d_model;
   prof_begin(HSTU_K_PROJ_IN_BWD, s);
   GemmArgs a;
@@ -305,6 +311,7 @@ hstu_status do_proj_in_bwd(const hstu_config* c, const void* W1, const void* x, 
   a.M = T; a.N = d; a.K = 4 * d;
   a.epi = dy ? EPI_RESID : EPI_STORE; a.C = dx; a.ldc = d; a.R = dy; a.ldr = d;
   a.io_f32 = c->io_dtype == HSTU_F32;
+  if (dy && a.io_f32 && c->dtype == HSTU_BF16) a.C2 = dx_low;
   cudaError_t e = cudaSuccess;
   // dW1 first: dx may alias dy but never x or dpre
   if (dW1) {
@@ -724,6 +731,15 @@ hstu_status hstu_fwd(const hstu_config* cfg, const hstu_weights* w, const void* 
                      const int64_t* seq_offsets, int32_t B, int64_t T, const int64_t* timestamps,
                      const int32_t* num_targets, void* y, void* saved, void* kv_out,
                      void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  return hstu_fwd_chain(cfg, w, x, nullptr, seq_offsets, B, T, timestamps, num_targets, y,
+                        nullptr, saved, kv_out, workspace, ws_bytes, stream);
+}
+
+hstu_status hstu_fwd_chain(const hstu_config* cfg, const hstu_weights* w, const void* x,
+                           const void* x_low, const int64_t* seq_offsets, int32_t B, int64_t T,
+                           const int64_t* timestamps, const int32_t* num_targets, void* y,
+                           void* y_low, void* saved, void* kv_out, void* workspace,
+                           size_t ws_bytes, cudaStream_t stream) {
   HSTU_TRY(check_cfg(cfg));
   HSTU_TRY(check_jagged(seq_offsets, B, T, timestamps, num_targets));
   HSTU_TRY(check_weights(cfg, w, true, true));
@@ -731,6 +747,10 @@ hstu_status hstu_fwd(const hstu_config* cfg, const hstu_weights* w, const void* 
   HSTU_TRY(need(y, T));
   HSTU_TRY(opt(saved));
   HSTU_TRY(opt(kv_out));
+  HSTU_TRY(opt(x_low));
+  HSTU_TRY(opt(y_low));
+  const bool lowio = cfg->io_dtype != cfg->dtype;   // fp32 residual stream, bf16 operands
+  if (!lowio) x_low = y_low = nullptr;
   const FwdWs L = fwd_ws(cfg, B, T);
   if (ws_bytes < L.total) return HSTU_ERR_WORKSPACE;
   if (T == 0 || B == 0) return HSTU_OK;
@@ -754,14 +774,27 @@ hstu_status hstu_fwd(const hstu_config* cfg, const hstu_weights* w, const void* 
     z = at(workspace, L.z);
   }
   const void* xop = nullptr;
-  HSTU_TRY(to_operand(cfg, x, T, xlow, &xop, stream));
+  if (x_low) {
+    // the bf16 copy of x came with the call; the saved block keeps its own
+    // copy for the backward unless x_low already is that part of it
+    xop = x_low;
+    if (saved && x_low != xlow) {
+      prof_begin(HSTU_K_MISC, stream);
+      cudaError_t e = cudaMemcpyAsync(xlow, x_low, (size_t)T * d * es, cudaMemcpyDeviceToDevice,
+                                      stream);
+      prof_end(HSTU_K_MISC, stream);
+      if (e != cudaSuccess) return HSTU_ERR_CUDA;
+    }
+  } else {
+    HSTU_TRY(to_operand(cfg, x, T, xlow, &xop, stream));
+  }
   HSTU_TRY(do_proj_in(cfg, w->W1, w->b1, xop, T, pre, g, stream));
   AttnArgs a = full_attn_args(cfg, w->rab_pos, w->rab_time, g, seq_offsets, B, T, timestamps,
                               num_targets, o);
   HSTU_TRY(do_attention_fwd(cfg, a, at(workspace, L.attn), ws_bytes - L.attn, stream,
                             HSTU_K_ATTN_FWD));
   HSTU_TRY(do_ln_fwd(cfg, w->ln_gamma, w->ln_beta, o, g, T, z, mean, rstd, stream));
-  HSTU_TRY(do_proj_out(cfg, w->W2, w->b2, z, x, T, y, stream));
+  HSTU_TRY(do_proj_out(cfg, w->W2, w->b2, z, x, T, y, stream, y_low));
   if (kv_out) {
     prof_begin(HSTU_K_MISC, stream);
     cudaError_t e = copy_columns(cfg->dtype, at(g, (size_t)d * es), 4 * d, kv_out, 2 * d, T, d,
@@ -820,9 +853,22 @@ hstu_status hstu_bwd(const hstu_config* cfg, const hstu_weights* w, const void* 
                      const int64_t* timestamps, const int32_t* num_targets, void* dx,
                      const hstu_grads* grads, void* workspace, size_t ws_bytes,
                      cudaStream_t stream) {
+  return hstu_bwd_chain(cfg, w, x, dy, nullptr, saved, seq_offsets, B, T, timestamps,
+                        num_targets, dx, nullptr, grads, workspace, ws_bytes, stream);
+}
+
+hstu_status hstu_bwd_chain(const hstu_config* cfg, const hstu_weights* w, const void* x,
+                           const void* dy, const void* dy_low, const void* saved,
+                           const int64_t* seq_offsets, int32_t B, int64_t T,
+                           const int64_t* timestamps, const int32_t* num_targets, void* dx,
+                           void* dx_low, const hstu_grads* grads, void* workspace,
+                           size_t ws_bytes, cudaStream_t stream) {
   HSTU_TRY(check_cfg(cfg));
   HSTU_TRY(check_jagged(seq_offsets, B, T, timestamps, num_targets));
   HSTU_TRY(check_weights(cfg, w, true, true));
+  HSTU_TRY(opt(dy_low));
+  HSTU_TRY(opt(dx_low));
+  if (cfg->io_dtype == cfg->dtype) dy_low = dx_low = nullptr;
   HSTU_TRY(need(x, T));
   HSTU_TRY(need(dy, T));
   HSTU_TRY(need(saved, T));
@@ -850,15 +896,15 @@ hstu_status hstu_bwd(const hstu_config* cfg, const hstu_weights* w, const void* 
   void* dpre = at(workspace, L.dpre);
   float* dq = reinterpret_cast<float*>(at(workspace, L.dq));
   const void* xop = cfg->io_dtype == cfg->dtype ? x : at(svd, off[HSTU_SAVED_XLOW]);
-  const void* dyop = nullptr;
-  HSTU_TRY(to_operand(cfg, dy, T, at(workspace, L.dylow), &dyop, stream));
+  const void* dyop = dy_low;
+  if (!dyop) HSTU_TRY(to_operand(cfg, dy, T, at(workspace, L.dylow), &dyop, stream));
   HSTU_TRY(do_proj_out_bwd(cfg, w->W2, z, dyop, T, dz, gr.dW2, gr.db2, stream));
   HSTU_TRY(do_ln_bwd(cfg, w->ln_gamma, w->ln_beta, dz, o, g, pre, mean, rstd, T, dO, dpre,
                      gr.dgamma, gr.dbeta, stream));
   HSTU_TRY(do_attention_bwd(cfg, w->rab_pos, w->rab_time, g, pre, dO, seq_offsets, B, T,
                             timestamps, num_targets, dpre, gr.drab_pos, gr.drab_time, dq,
                             at(workspace, L.attn), ws_bytes - L.attn, stream));
-  HSTU_TRY(do_proj_in_bwd(cfg, w->W1, xop, dpre, dy, T, dx, gr.dW1, gr.db1, stream));
+  HSTU_TRY(do_proj_in_bwd(cfg, w->W1, xop, dpre, dy, T, dx, gr.dW1, gr.db1, stream, dx_low));
   return HSTU_OK;
 }
 

@@ -10,6 +10,15 @@ cudaError_t attention_bwd_simt(int dtype, const AttnBwdArgs& a, cudaStream_t s);
 
 cudaError_t gemm(int dtype, const GemmArgs& g, cudaStream_t s) {
   if (gemm_tc_supported(dtype, g)) return gemm_tc(g, device_status(), s);
+  if (g.epi == EPI_RESID && g.io_f32 && g.C2) {
+    // the CUDA-core GEMM writes C only; its bf16 copy follows
+    GemmArgs h = g;
+    h.C2 = nullptr;
+    cudaError_t e = gemm_simt(dtype, h, s);
+    if (e != cudaSuccess) return e;
+    if (g.ldc != g.N) return cudaErrorInvalidValue;   // the layers' rows are dense
+    return convert_f32_to_bf16(static_cast<const float*>(g.C), g.C2, g.M * g.N, s);
+  }
   return gemm_simt(dtype, g, s);
 }
 

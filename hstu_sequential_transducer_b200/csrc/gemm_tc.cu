@@ -71,6 +71,8 @@ struct KParams {
   const void* bias;     // [N] bf16 or null
   uint32_t* status;
   bool has_c;           // SILU_SPLIT: write Pre too
+  void* c2;             // RESID with fp32 output: also a bf16 copy of C here (or null)
+  int64_t ldc2;
 };
 
 // SiLU(x) = h + h tanh(h) with h = x / 2 (x sigmoid(x), as an identity).
@@ -374,14 +376,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(wstg + sw128(row, j)) = o;
           }
         } else {
+          uint32_t lo[16];   // RESID: the chunk's row rounded to bf16 for the copy in c2
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             if (EPI == EPI_RESID) {
               const float4 rr = *reinterpret_cast<const float4*>(wstg + sw128(row, j));
               o.x += rr.x; o.y += rr.y; o.z += rr.z; o.w += rr.w;
+              lo[2 * j] = pack_bf16(o.x, o.y);
+              lo[2 * j + 1] = pack_bf16(o.z, o.w);
             }
             *reinterpret_cast<float4*>(wstg + sw128(row, j)) = o;
+          }
+          if (EPI == EPI_RESID && p.c2 != nullptr && m0 + row < p.M) {
+            // 16-byte pieces straight to global (N is a multiple of 16, so a
+            // piece of 8 columns is wholly inside or outside the matrix)
+            bf16* dst = static_cast<bf16*>(p.c2) + (int64_t)(m0 + row) * p.ldc2 + n0 + c0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (n0 + c0 + 8 * q < p.N)
+                *reinterpret_cast<uint4*>(dst + 8 * q) =
+                    make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
           }
         }
         fence_proxy_async_smem();
@@ -483,6 +498,8 @@ cudaError_t run_cfg(const GemmArgs& g, uint32_t* status, cudaStream_t s) {
   p.bias = g.bias;
   p.status = status;
   p.has_c = g.C != nullptr;
+  p.c2 = (EPI == EPI_RESID && o32) ? g.C2 : nullptr;
+  p.ldc2 = g.ldc;
   const int units = p.tiles * p.ksplit;
   auto kern = gemm_tc_kernel<BN, AK, BKM, EPI, TOUT, PAIR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);

@@ -31,7 +31,8 @@ struct GemmArgs {
   int64_t M = 0, N = 0, K = 0;
   int epi = EPI_STORE;
   void* C = nullptr;        // dtype output (row-major, ldc)
-  void* C2 = nullptr;       // second dtype output (EPI_SILU_SPLIT)
+  void* C2 = nullptr;       // second output: G (EPI_SILU_SPLIT); a bf16 copy of the fp32 C
+                            // (EPI_RESID with io_f32; row stride ldc)
   int64_t ldc = 0;
   const void* bias = nullptr;  // [N] dtype
   const void* R = nullptr;     // residual, row-major ldr (EPI_RESID)

@@ -79,6 +79,8 @@ _SIGS = {
     "hstu_fwd": (I32, [_CP, _WP, P, P, I32, I64, P, P, P, P, P, P, S, P]),
     "hstu_fwd_cached": (I32, [_CP, _WP, P, P, I32, I64, P, P, P, I64, P, P, P, S, P]),
     "hstu_bwd": (I32, [_CP, _WP, P, P, P, P, I32, I64, P, P, P, _GP, P, S, P]),
+    "hstu_fwd_chain": (I32, [_CP, _WP, P, P, P, I32, I64, P, P, P, P, P, P, P, S, P]),
+    "hstu_bwd_chain": (I32, [_CP, _WP, P, P, P, P, P, I32, I64, P, P, P, P, _GP, P, S, P]),
     "hstu_validate_inputs": (I32, [P, I32, I64, P, P, I32, P, P]),
     "hstu_sl_subsequence_length": (I64, [I64, c_double]),
     "hstu_stochastic_length": (I32, [P, P, I32, I64, I64, P, P, P, P, P]),
@@ -411,17 +413,25 @@ def gather_rows(src, gather_index, d_num_rows, out, stream=None):
 # ----------------------------------------------------------------------------
 
 def fwd(cfg, w: LayerWeights, x, offsets, timestamps, num_targets=None, y=None, saved=None,
-        kv_out=None, stream=None):
+        kv_out=None, stream=None, x_low=None, y_low=None):
     """One layer forward; returns y.  `saved` (uint8, saved_bytes) is filled
-    for a later bwd() when given."""
+    for a later bwd() when given.  x_low / y_low (bf16 [T][d] buffers, fp32
+    io only): the bf16 copy of x from the previous layer, and where to write
+    the bf16 copy of y for the next one (hstu_fwd_chain)."""
     B, T = offsets.numel() - 1, x.shape[0]
     ws_n, _ = workspace_size(cfg, B, T)
     ws = workspace(ws_n, x.device)
     if y is None:
         y = torch.empty_like(x)
-    _check(lib().hstu_fwd(ctypes.byref(cfg), ctypes.byref(w.c()), ptr(x), ptr(offsets), B, T,
-                          ptr(timestamps), ptr(num_targets), ptr(y), ptr(saved), ptr(kv_out),
-                          ptr(ws), ws.numel(), stream_ptr(stream)), "hstu_fwd")
+    if x_low is None and y_low is None:
+        _check(lib().hstu_fwd(ctypes.byref(cfg), ctypes.byref(w.c()), ptr(x), ptr(offsets), B, T,
+                              ptr(timestamps), ptr(num_targets), ptr(y), ptr(saved), ptr(kv_out),
+                              ptr(ws), ws.numel(), stream_ptr(stream)), "hstu_fwd")
+    else:
+        _check(lib().hstu_fwd_chain(ctypes.byref(cfg), ctypes.byref(w.c()), ptr(x), ptr(x_low),
+                                    ptr(offsets), B, T, ptr(timestamps), ptr(num_targets), ptr(y),
+                                    ptr(y_low), ptr(saved), ptr(kv_out), ptr(ws), ws.numel(),
+                                    stream_ptr(stream)), "hstu_fwd_chain")
     return y
 
 
@@ -440,16 +450,25 @@ def fwd_cached(cfg, w: LayerWeights, cand_x, cand_offsets, cand_ts, hist_kv, his
 
 
 def bwd(cfg, w: LayerWeights, x, dy, saved, offsets, timestamps, num_targets=None, dx=None,
-        grads: Optional[LayerGradBufs] = None, stream=None):
+        grads: Optional[LayerGradBufs] = None, stream=None, dy_low=None, dx_low=None):
+    """One layer backward; returns dx.  dy_low / dx_low (bf16 [T][d], fp32 io
+    only): the bf16 copy of dy from the layer above, and where to write the
+    bf16 copy of dx for the layer below (hstu_bwd_chain)."""
     B, T = offsets.numel() - 1, x.shape[0]
     ws_n, _ = workspace_size(cfg, B, T)
     ws = workspace(ws_n, x.device)
     if dx is None:
         dx = torch.empty_like(x)
     g = grads.c() if grads is not None else Grads()
-    _check(lib().hstu_bwd(ctypes.byref(cfg), ctypes.byref(w.c()), ptr(x), ptr(dy), ptr(saved),
-                          ptr(offsets), B, T, ptr(timestamps), ptr(num_targets), ptr(dx),
-                          ctypes.byref(g), ptr(ws), ws.numel(), stream_ptr(stream)), "hstu_bwd")
+    if dy_low is None and dx_low is None:
+        _check(lib().hstu_bwd(ctypes.byref(cfg), ctypes.byref(w.c()), ptr(x), ptr(dy), ptr(saved),
+                              ptr(offsets), B, T, ptr(timestamps), ptr(num_targets), ptr(dx),
+                              ctypes.byref(g), ptr(ws), ws.numel(), stream_ptr(stream)), "hstu_bwd")
+    else:
+        _check(lib().hstu_bwd_chain(ctypes.byref(cfg), ctypes.byref(w.c()), ptr(x), ptr(dy),
+                                    ptr(dy_low), ptr(saved), ptr(offsets), B, T, ptr(timestamps),
+                                    ptr(num_targets), ptr(dx), ptr(dx_low), ctypes.byref(g),
+                                    ptr(ws), ws.numel(), stream_ptr(stream)), "hstu_bwd_chain")
     return dx
 
 

@@ -66,18 +66,31 @@ class DeviceWorkload:
         return self.x.shape[0]
 
 
-def forward_stack(dw: DeviceWorkload, num_layers: Optional[int] = None, stream=None):
-    """Inference forward through the stack; returns the last layer's output."""
+def forward_stack(dw: DeviceWorkload, num_layers: Optional[int] = None, stream=None,
+                  chain: bool = True):
+    """Inference forward through the stack; returns the last layer's output.
+    With an fp32 residual stream and bf16 operands, each layer's output
+    epilogue also writes the bf16 copy the next layer reads (two alternating
+    buffers) unless chain is False."""
     y = dw.x
-    for w in dw.layers[:num_layers]:
-        y = H.fwd(dw.cfg, w, y, dw.offsets, dw.timestamps, dw.num_targets, stream=stream)
+    layers = dw.layers[:num_layers]
+    n = len(layers)
+    ch = chain and dw.cfg.io_dtype != dw.cfg.dtype and n > 1
+    lo = []
+    if ch:
+        lt = H.torch_dtype(dw.cfg.dtype)
+        lo = [torch.empty(dw.T, dw.cfg.d_model, dtype=lt, device=dw.x.device) for _ in range(2)]
+    for i, w in enumerate(layers):
+        y = H.fwd(dw.cfg, w, y, dw.offsets, dw.timestamps, dw.num_targets, stream=stream,
+                  x_low=lo[i % 2] if ch and i > 0 else None,
+                  y_low=lo[(i + 1) % 2] if ch and i + 1 < n else None)
     return y
 
 
 class TrainStep:
     """Buffers for a forward+backward step over the whole stack, allocated once."""
 
-    def __init__(self, dw: DeviceWorkload):
+    def __init__(self, dw: DeviceWorkload, chain: bool = True):
         self.dw = dw
         T = dw.T
         _, saved_n = H.workspace_size(dw.cfg, dw.B, T)
@@ -85,6 +98,16 @@ class TrainStep:
         self.saved = [torch.empty(saved_n, dtype=torch.uint8, device=dev) for _ in dw.layers]
         self.acts = [dw.x] + [torch.empty_like(dw.x) for _ in dw.layers]
         self.gbuf = [torch.empty_like(dw.x), torch.empty_like(dw.x)]
+        # fp32 residual stream with bf16 operands: each layer's output epilogue
+        # also writes the bf16 copy the next layer reads (forward: straight
+        # into that layer's saved block; backward: two alternating buffers)
+        self.chain = chain and dw.cfg.io_dtype != dw.cfg.dtype
+        self.xlow = []
+        self.dlow = []
+        if self.chain:
+            self.xlow = [H.saved_views(dw.cfg, sv, T)["xlow"] for sv in self.saved]
+            lt = H.torch_dtype(dw.cfg.dtype)
+            self.dlow = [torch.empty(T, dw.cfg.d_model, dtype=lt, device=dev) for _ in range(2)]
         # every layer's fp32 gradients are views of one flat buffer (one
         # all-reduce in data-parallel training)
         names = ("W1", "W2", "b1", "b2", "ln_gamma", "ln_beta", "rab_pos", "rab_time")
@@ -121,14 +144,20 @@ class TrainStep:
         backward has been issued (layers in reverse order), e.g. to start the
         all-reduce of that layer's gradients."""
         dw = self.dw
+        L = len(dw.layers)
+        ch = self.chain
         for i, w in enumerate(dw.layers):
             H.fwd(dw.cfg, w, self.acts[i], dw.offsets, dw.timestamps, dw.num_targets,
-                  y=self.acts[i + 1], saved=self.saved[i], stream=stream)
+                  y=self.acts[i + 1], saved=self.saved[i], stream=stream,
+                  x_low=self.xlow[i] if ch and i > 0 else None,
+                  y_low=self.xlow[i + 1] if ch and i + 1 < L else None)
         g = dw.dy if dy is None else dy
-        for i in range(len(dw.layers) - 1, -1, -1):
+        for i in range(L - 1, -1, -1):
             out = self.gbuf[i % 2]
             H.bwd(dw.cfg, dw.layers[i], self.acts[i], g, self.saved[i], dw.offsets, dw.timestamps,
-                  dw.num_targets, dx=out, grads=self.grads[i], stream=stream)
+                  dw.num_targets, dx=out, grads=self.grads[i], stream=stream,
+                  dy_low=self.dlow[(i + 1) % 2] if ch and i < L - 1 else None,
+                  dx_low=self.dlow[i % 2] if ch and i > 0 else None)
             if on_layer_grads is not None:
                 on_layer_grads(i)
             g = out

@@ -309,6 +309,25 @@ hstu_status hstu_fwd(const hstu_config* cfg, const hstu_weights* w, const void* 
                      void* saved, void* kv_out, void* workspace, size_t ws_bytes,
                      cudaStream_t stream);
 
+/* hstu_fwd for a layer inside a stack whose residual stream is fp32
+ * (io_dtype HSTU_F32) and whose operands are bf16 (dtype HSTU_BF16): the
+ * bf16 copy of each layer's input, which the W1 projection reads, comes from
+ * the previous layer's output epilogue instead of a separate conversion.
+ *   x_low: NULL, or [T][d] bf16 already holding x rounded to bf16 (the
+ *          previous layer's y_low).  With `saved`, the backward needs that
+ *          copy inside the saved block: pass the block's HSTU_SAVED_XLOW part
+ *          (hstu_saved_layout) to avoid a copy, else it is copied there.
+ *   y_low: NULL, or [T][d] bf16 receiving y rounded to bf16 by the W2
+ *          projection's epilogue (e.g. the next layer's saved XLOW part).  It
+ *          must not overlap x, x_low, y or this layer's saved block.
+ * Both are ignored when io_dtype equals dtype.  The results are those of
+ * hstu_fwd bit for bit (the same rounding of the same fp32 values). */
+hstu_status hstu_fwd_chain(const hstu_config* cfg, const hstu_weights* w, const void* x,
+                           const void* x_low, const int64_t* seq_offsets, int32_t B, int64_t T,
+                           const int64_t* timestamps, const int32_t* num_targets, void* y,
+                           void* y_low, void* saved, void* kv_out, void* workspace,
+                           size_t ws_bytes, cudaStream_t stream);
+
 /* One layer forward of M-FALCON candidates against a cached history (see
  * hstu_attention_fwd_cached for the layouts).  cand_x, y [Tc][d] in
  * cfg->io_dtype; hist_kv in cfg->dtype. */
@@ -328,6 +347,22 @@ hstu_status hstu_bwd(const hstu_config* cfg, const hstu_weights* w, const void* 
                      int32_t B, int64_t T, const int64_t* timestamps,
                      const int32_t* num_targets, void* dx, const hstu_grads* grads,
                      void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* hstu_bwd inside a stack (fp32 io, bf16 operands, as hstu_fwd_chain):
+ *   dy_low: NULL, or [T][d] bf16 already holding dy rounded to bf16 (the
+ *           layer above's dx_low); used as the dY operand of the W2
+ *           gradients instead of converting dy.
+ *   dx_low: NULL, or [T][d] bf16 receiving dx rounded to bf16 by the dX
+ *           epilogue, for the layer below.  It may alias dy_low (which is
+ *           read before dx is formed) but no other argument.
+ * Both are ignored when io_dtype equals dtype; results equal hstu_bwd's bit
+ * for bit. */
+hstu_status hstu_bwd_chain(const hstu_config* cfg, const hstu_weights* w, const void* x,
+                           const void* dy, const void* dy_low, const void* saved,
+                           const int64_t* seq_offsets, int32_t B, int64_t T,
+                           const int64_t* timestamps, const int32_t* num_targets, void* dx,
+                           void* dx_low, const hstu_grads* grads, void* workspace,
+                           size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Stochastic Length (training-input subsampling)                            */

@@ -92,6 +92,18 @@ def test_host_argument_errors_return_before_launch(L):
     # negative sizes
     assert L.hstu_ln_gate_fwd(ctypes.byref(c), None, None, None, None, -1, None, None, None,
                               None) == 1
+    # the chained layer calls: a misaligned bf16 copy is refused, a short
+    # workspace too, before any launch
+    st = L.hstu_fwd_chain(ctypes.byref(c), ctypes.byref(w), 0x2000, 0x7001, ctypes.addressof(off),
+                          2, 10, 0x4000, None, 0x5000, None, None, None, 0x6000, 1 << 30, None)
+    assert st == 2
+    st = L.hstu_fwd_chain(ctypes.byref(c), ctypes.byref(w), 0x2000, 0x7000, ctypes.addressof(off),
+                          2, 10, 0x4000, None, 0x5000, 0x8000, None, None, 0x6000, 16, None)
+    assert st == 4
+    st = L.hstu_bwd_chain(ctypes.byref(c), ctypes.byref(w), 0x2000, 0x3000, 0x7000, 0x9000,
+                          ctypes.addressof(off), 2, 10, 0x4000, None, 0x5000, 0x8001, None,
+                          0x6000, 1 << 30, None)
+    assert st == 2
 
 
 def test_sl_subsequence_length_host(L):

@@ -620,6 +620,45 @@ def test_training_subset_fwd_bwd_bf16(training_oracle):
             check_grad(np_(got), ref, "bf16", f"layer {li} {name}", deep=True)
 
 
+def test_chained_layers_match_separate_conversions():
+    """hstu_fwd_chain / hstu_bwd_chain: each layer's output epilogue also
+    writes the bf16 copy of its fp32 output that the next layer reads, in
+    place of a conversion kernel at the start of that layer.  The forward is
+    bit-identical to the unchained calls, every bf16 copy equals the rounded
+    fp32 tensor exactly, dX agrees up to the ordering of the backward's fp32
+    reductions, and 2 (L - 1) conversion launches go away."""
+    L = 3
+    w = W.custom([300, 1, 129, 64, 257, 700], d=256, H=2, dtype="bf16", layers=L, N=700.0,
+                 backward=True, seed=77)
+    dw = S.DeviceWorkload.from_workload(w)
+    res = {}
+    for chain in (False, True):
+        step = S.TrainStep(dw, chain=chain)
+        assert step.chain == chain
+        step.zero_grads()
+        torch.cuda.synchronize()
+        n0 = H.launch_count()
+        dx = step.run()
+        torch.cuda.synchronize()
+        res[chain] = (step, dx.clone(), H.launch_count() - n0)
+        assert H.device_status() == 0
+    s0, dx0, n_plain = res[False]
+    s1, dx1, n_chain = res[True]
+    assert n_plain - n_chain == 2 * (L - 1)
+    for i in range(1, L + 1):
+        assert torch.equal(s0.acts[i], s1.acts[i]), f"layer {i - 1} output"
+    for i in range(L):       # the saved bf16 operand of every layer, chained or converted
+        xl = H.saved_views(dw.cfg, s1.saved[i], dw.T)["xlow"]
+        assert torch.equal(xl, s1.acts[i].to(torch.bfloat16)), f"layer {i} saved x (bf16)"
+    # layer 1 wrote its dX (gbuf[1]) and the bf16 copy for layer 0 (dlow[1])
+    assert torch.equal(s1.dlow[1], s1.gbuf[1].to(torch.bfloat16))
+    check_el(np_(dx1), np_(dx0).astype(np.float64), "bf16", "dX chained vs separate")
+    y0 = S.forward_stack(dw, chain=False)
+    y1 = S.forward_stack(dw, chain=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+
+
 def test_training_full_size_sampled(training_oracle):
     """The full training workload (64 sequences, 8 layers, fwd+bwd) in the
     launch configuration the benchmark times; Y and dX rows of the two sampled

@@ -6,6 +6,9 @@
 #include <mutex>
 #include <vector>
 #include <atomic>
+#include <cstdlib>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -27,6 +30,18 @@ std::vector<ProfRecord> g_prof_records;
 std::vector<cudaEvent_t> g_event_pool;
 std::vector<std::pair<int, cudaEvent_t>> g_open;  // started, not yet stopped
 std::atomic<int64_t> g_launches{0};
+
+// NVTX ranges around the same regions as the profiler's events, named after
+// the kernel class, for NVTX-aware tracers; off unless HSTU_NVTX=1 or
+// hstu_nvtx_enable(1).
+bool nvtx_env() {
+  const char* v = std::getenv("HSTU_NVTX");
+  return v && v[0] == '1';
+}
+std::atomic<bool> g_nvtx{nvtx_env()};
+const char* const kClassNames[HSTU_K_COUNT] = {
+    "proj_in", "attn_fwd", "ln_fwd", "proj_out", "proj_out_bwd", "ln_bwd",
+    "attn_bwd", "proj_in_bwd", "attn_cached", "misc", "softmax_fwd"};
 
 cudaEvent_t take_event() {
   if (!g_event_pool.empty()) {
@@ -386,6 +401,8 @@ uint32_t* device_status() {
 }
 
 void prof_begin(int id, cudaStream_t s) {
+  if (g_nvtx.load(std::memory_order_relaxed) && id >= 0 && id < HSTU_K_COUNT)
+    nvtxRangePushA(kClassNames[id]);
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (!g_prof_on) return;
   cudaEvent_t e = take_event();
@@ -395,6 +412,7 @@ void prof_begin(int id, cudaStream_t s) {
 }
 
 void prof_end(int id, cudaStream_t s) {
+  if (g_nvtx.load(std::memory_order_relaxed) && id >= 0 && id < HSTU_K_COUNT) nvtxRangePop();
   std::lock_guard<std::mutex> lk(g_prof_mu);
   if (!g_prof_on) return;
   for (size_t i = g_open.size(); i-- > 0;) {
@@ -429,6 +447,8 @@ const char* hstu_status_string(hstu_status s) {
 }
 
 const char* hstu_version(void) { return "hstu-b200 0.1 (sm_100a)"; }
+
+void hstu_nvtx_enable(int32_t on) { g_nvtx.store(on != 0, std::memory_order_relaxed); }
 
 void hstu_profiler_enable(int32_t on) {
   std::lock_guard<std::mutex> lk(g_prof_mu);

@@ -86,6 +86,7 @@ _SIGS = {
     "hstu_stochastic_length": (I32, [P, P, I32, I64, I64, P, P, P, P, P]),
     "hstu_gather_rows": (I32, [P, I64, I64, P, P, I64, I64, P, I64, P]),
     "hstu_profiler_enable": (None, [I32]),
+    "hstu_nvtx_enable": (None, [I32]),
     "hstu_profiler_collect": (I32, [I32, POINTER(c_int64), POINTER(c_double)]),
     "hstu_profiler_reset": (None, []),
     "hstu_launch_count": (I64, []),
@@ -478,6 +479,11 @@ def bwd(cfg, w: LayerWeights, x, dy, saved, offsets, timestamps, num_targets=Non
 
 def profiler_enable(on: bool = True):
     lib().hstu_profiler_enable(1 if on else 0)
+
+
+def nvtx_enable(on: bool = True):
+    """NVTX ranges named after the kernel classes around the library's steps."""
+    lib().hstu_nvtx_enable(1 if on else 0)
 
 
 def profiler_reset():

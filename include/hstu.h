@@ -439,6 +439,15 @@ typedef enum {
 } hstu_kernel_id;
 
 void hstu_profiler_enable(int32_t on);
+/* NVTX ranges: while on, each of those regions is also an NVTX push/pop
+ * range on the calling host thread, named after its kernel class
+ * ("proj_in", "attn_fwd", "ln_fwd", "proj_out", "proj_out_bwd", "ln_bwd",
+ * "attn_bwd", "proj_in_bwd", "attn_cached", "misc", "softmax_fwd"), so that an
+ * NVTX-aware tracer or `ncu --nvtx` can select the library's steps.  Off by
+ * default; the environment variable HSTU_NVTX=1 turns it on when the library
+ * loads.  A switch flipped between a region's begin and end leaves that one
+ * range unbalanced: flip it between calls. */
+void hstu_nvtx_enable(int32_t on);
 /* Waits for the recorded events, then returns launches and total milliseconds
  * of kernel class `id` since the last reset. */
 hstu_status hstu_profiler_collect(int32_t id, int64_t* launches, double* total_ms);

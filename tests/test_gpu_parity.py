@@ -659,6 +659,22 @@ def test_chained_layers_match_separate_conversions():
     assert torch.equal(y0, y1)
 
 
+def test_nvtx_ranges_leave_results_unchanged():
+    """With NVTX ranges on (hstu_nvtx_enable), a stack forward gives the same
+    bits as with them off; the ranges only mark the host timeline."""
+    w = W.custom([300, 129, 64], d=256, H=2, dtype="bf16", layers=2, N=300.0, seed=78)
+    dw = S.DeviceWorkload.from_workload(w)
+    y0 = S.forward_stack(dw).clone()
+    H.nvtx_enable(True)
+    try:
+        y1 = S.forward_stack(dw).clone()
+    finally:
+        H.nvtx_enable(False)
+    torch.cuda.synchronize()
+    assert H.device_status() == 0
+    assert torch.equal(y0, y1)
+
+
 def test_training_full_size_sampled(training_oracle):
     """The full training workload (64 sequences, 8 layers, fwd+bwd) in the
     launch configuration the benchmark times; Y and dX rows of the two sampled

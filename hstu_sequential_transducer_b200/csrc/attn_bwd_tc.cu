@@ -356,7 +356,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         for (int u = 0; u < 4; ++u) {
           const int c = lane + 32 * u;
           // past the sequence: a large sentinel keeps the staged times sorted
-          qts[c] = (q0 + c < n) ? a.q_ts[s0 + q0 + c] : (1LL << 62);
+          qts[c] = (q0 + c < n && bounds_ok(s0 + q0 + c < a.q_rows, P.status))
+                    ? a.q_ts[s0 + q0 + c] : (1LL << 62);
         }
         __syncwarp();
         if (lane == 0) {
@@ -462,7 +463,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       const int k0 = item.kt * kT;
       const int nqt = bcost(n, item.kt);
       const int jk = k0 + row;                       // key index in the sequence
-      const bool kvalid = jk < hlen;
+      const bool kvalid = jk < hlen && bounds_ok(s0 + jk < a.kv_rows, P.status);
       const long long tk = kvalid ? a.kv_ts[s0 + jk] : 0;
       if (item.h != cur_h) {
         named_barrier(1, kAct);
@@ -619,7 +620,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
           uint32_t r[32];
           tmem_ld32(tA + lane_off + c * 32, r);
           tmem_ld_wait();
-          if (qrow < n) {
+          if (qrow < n && bounds_ok(s0 + qrow < a.q_rows, P.status)) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
               red_add_v4(dq + c * 32 + i, __uint_as_float(r[i]) * inv_N, __uint_as_float(r[i + 1]) * inv_N,
@@ -880,7 +881,7 @@ __global__ void __launch_bounds__(kB3Threads, 1)
           tma_prefetch_2d(tm, item.h * DH + 64 * (lane & 1), (int32_t)(s0 + qp));
         } else if (lane < 9) {
           const int r = qp + (lane - 4) * 16;       // 16 times of 8 bytes per 128-byte line
-          if (r < n) prefetch_l2(a.q_ts + s0 + r);
+          if (r < n && bounds_ok(s0 + r < a.q_rows, P.status)) prefetch_l2(a.q_ts + s0 + r);
         }
       };
       for (int mp = 1; mp < kPrefetch; ++mp) prefetch(mp);
@@ -897,7 +898,8 @@ __global__ void __launch_bounds__(kB3Threads, 1)
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int c = lane + 32 * u;
-          tq[u] = (q0 + c < n) ? a.q_ts[s0 + q0 + c] : (1LL << 62);
+          tq[u] = (q0 + c < n && bounds_ok(s0 + q0 + c < a.q_rows, P.status))
+                    ? a.q_ts[s0 + q0 + c] : (1LL << 62);
         }
         if (lane == 0) ok = mbar_wait(&qd_empty[st], par ^ 1, abort_flag, P.status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -1060,7 +1062,7 @@ __global__ void __launch_bounds__(kB3Threads, 1)
       tc_fence_after();
       {
         const int jk = k0 + row;
-        const bool kvalid = jk < hlen;
+        const bool kvalid = jk < hlen && bounds_ok(s0 + jk < a.kv_rows, P.status);
         const bf16* pre = static_cast<const bf16*>(P.A.pre);
         bf16* dpre = static_cast<bf16*>(P.A.dpre);
         const int d = P.A.d;
@@ -1133,7 +1135,7 @@ __global__ void __launch_bounds__(kB3Threads, 1)
       const int k0 = item.kt * kT;
       const int nqb = qblocks(n, item.kt);
       const int jk = k0 + row;
-      const bool kvalid = jk < hlen;
+      const bool kvalid = jk < hlen && bounds_ok(s0 + jk < a.kv_rows, P.status);
       const long long tk = kvalid ? a.kv_ts[s0 + jk] : 0;
       if (item.h != cur_h) {
         named_barrier(bid, 128);

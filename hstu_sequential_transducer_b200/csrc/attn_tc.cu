@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(352, 1)
           tma_prefetch_2d(&tmK, item.h * DH + 64 * lane, (int32_t)(g.ks + kp));
         } else if (lane >= 8 && lane < 16) {
           const int r = kp + (lane - 8) * 16;          // 16 times per 128-byte line
-          if (r < kend) prefetch_l2(a.kv_ts + g.ks + r);
+          if (r < kend && bounds_ok(g.ks + r < a.kv_rows, P.status)) prefetch_l2(a.kv_ts + g.ks + r);
         }
       };
       for (int jp = 0; jp < C::PREFETCH; ++jp) prefetch(jp);
@@ -352,7 +352,8 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int c = lane + 32 * q;
-          tk[q] = (k0 + c < kend) ? a.kv_ts[g.ks + k0 + c] : (1LL << 62);
+          tk[q] = (k0 + c < kend && bounds_ok(g.ks + k0 + c < a.kv_rows, P.status))
+                      ? a.kv_ts[g.ks + k0 + c] : (1LL << 62);
         }
         const int tslot = (int)(n % C::TS_STAGES);
         const uint32_t tpar = (n / C::TS_STAGES) & 1;
@@ -505,7 +506,9 @@ __global__ void __launch_bounds__(352, 1)
       const int qpos = g.qbase + r0 + row;
       const int qp_clamped = min(qpos, g.hlen);
       const bool cand = qpos >= g.hlen;
-      const long long tq = rvalid ? a.q_ts[g.qs + r0 + row] : 0;
+      // rows of the query tensor this thread reads and writes directly
+      const bool row_in = !rvalid || bounds_ok(g.qs + r0 + row < a.q_rows, P.status);
+      const long long tq = rvalid && row_in ? a.q_ts[g.qs + r0 + row] : 0;
       if (item.h != cur_h) {
         named_barrier(bid, 128);
         const int t = (threadIdx.x - 64) & 127;
@@ -606,7 +609,7 @@ __global__ void __launch_bounds__(352, 1)
       float* O = static_cast<float*>(a.o);
       const int h = item.h;
       float self_w = 0.f;
-      if (cand && rvalid) {
+      if (cand && rvalid && row_in) {
         const bf16* q = static_cast<const bf16*>(a.q) + (g.qs + r0 + row) * a.q_stride + h * DH;
         const bf16* k = static_cast<const bf16*>(a.self_k) + (g.qs + r0 + row) * a.q_stride + h * DH;
         float sdot = 0.f;
@@ -648,7 +651,9 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
         }
-        if (rvalid) {
+        if (rvalid && row_in &&
+            bounds_ok(h * odh + c * 32 + 32 <= a.o_stride && h * DH + c * 32 + 32 <= a.q_stride,
+                      P.status)) {
           if (cand) {
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {

@@ -16,6 +16,22 @@ namespace tc {
 // Device status bits (ORed into the library's device status word).
 constexpr uint32_t kStatusTimeout = 0x100u;
 constexpr uint32_t kStatusSmemAlign = 0x200u;
+constexpr uint32_t kStatusBounds = 0x400u;
+
+// Index check of the debug build (-DHSTU_DEBUG) on a direct global access:
+// true when `ok`; otherwise ORs kStatusBounds into *status and returns false,
+// so that the caller skips the access instead of faulting (no trap).  The
+// release build compiles it to `true`.
+__device__ __forceinline__ bool bounds_ok(bool ok, uint32_t* status) {
+#ifdef HSTU_DEBUG
+  if (!ok && status) atomicOr(status, kStatusBounds);
+  return ok;
+#else
+  (void)ok;
+  (void)status;
+  return true;
+#endif
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -16,7 +16,10 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libhstu.so")
+# HSTU_DEBUG_BUILD=1 loads the debug build (-DHSTU_DEBUG: index checks on the
+# attention kernels' direct global accesses, reported as HSTU_DEVICE_BOUNDS)
+DEBUG_BUILD = os.environ.get("HSTU_DEBUG_BUILD") == "1"
+LIB_PATH = os.path.join(_HERE, "libhstu_debug.so" if DEBUG_BUILD else "libhstu.so")
 
 HSTU_F32, HSTU_BF16 = 0, 1
 SAVED_PRE, SAVED_G, SAVED_O, SAVED_Z, SAVED_MEAN, SAVED_RSTD, SAVED_XLOW, SAVED_COUNT = range(8)
@@ -103,7 +106,8 @@ def lib():
     if _lib is None:
         if not os.path.exists(LIB_PATH):
             raise RuntimeError(f"{LIB_PATH} is missing: run `python -m "
-                               "hstu_sequential_transducer_b200.build` first")
+                               "hstu_sequential_transducer_b200.build"
+                               f"{' --debug' if DEBUG_BUILD else ''}` first")
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in _SIGS.items():
             f = getattr(L, name)
@@ -516,7 +520,7 @@ def selftest_wait_timeout(limit_ns: int, result=None, stream=None):
            "hstu_selftest_wait_timeout")
 
 
-DEVICE_TIMEOUT, DEVICE_SMEM_ALIGN = 0x100, 0x200
+DEVICE_TIMEOUT, DEVICE_SMEM_ALIGN, DEVICE_BOUNDS = 0x100, 0x200, 0x400
 
 
 def version() -> str:

@@ -461,10 +461,14 @@ int64_t hstu_launch_count(void);
  * then abandoned its work and exited cleanly; its outputs are not valid);
  * bit HSTU_DEVICE_SMEM_ALIGN when a kernel that packs its whole shared-memory
  * budget found its dynamic shared memory not 1024-byte aligned (it exits at
- * once; outputs not valid).  Copies the word to *host_out, synchronising
- * `stream`; clears it when `clear` is non-zero. */
+ * once; outputs not valid); bit HSTU_DEVICE_BOUNDS, in the debug build only
+ * (libhstu_debug.so, compiled with -DHSTU_DEBUG), when an index check on a
+ * direct global access of an attention kernel failed (the access was skipped;
+ * outputs not valid).  Copies the word to *host_out, synchronising `stream`;
+ * clears it when `clear` is non-zero. */
 #define HSTU_DEVICE_TIMEOUT 0x100u
 #define HSTU_DEVICE_SMEM_ALIGN 0x200u
+#define HSTU_DEVICE_BOUNDS 0x400u
 hstu_status hstu_device_status(uint32_t* host_out, int32_t clear, cudaStream_t stream);
 
 /* Diagnostic of the bounded-wait path (the pages have no counterpart: this

@@ -659,6 +659,37 @@ def test_chained_layers_match_separate_conversions():
     assert torch.equal(y0, y1)
 
 
+def test_chained_calls_other_buffers():
+    """The chained calls with buffers other than the stack's: an x_low of its
+    own with a saved block (copied into the block's bf16 part, which the
+    backward reads) and dx_low aliasing dy_low (allowed: dy_low is read
+    before dx is formed).  Results as the unchained calls."""
+    w = W.custom([300, 129, 64], d=256, H=2, dtype="bf16", layers=1, N=300.0, backward=True,
+                 seed=79)
+    dw = S.DeviceWorkload.from_workload(w)
+    lw = dw.layers[0]
+    _, saved_n = H.workspace_size(dw.cfg, dw.B, dw.T)
+    sv0 = torch.empty(saved_n, dtype=torch.uint8, device=DEV)
+    sv1 = torch.empty(saved_n, dtype=torch.uint8, device=DEV)
+    y0 = H.fwd(dw.cfg, lw, dw.x, dw.offsets, dw.timestamps, None, saved=sv0)
+    x_low = dw.x.to(torch.bfloat16)
+    y_low = torch.full_like(x_low, float("nan"))
+    y1 = H.fwd(dw.cfg, lw, dw.x, dw.offsets, dw.timestamps, None, saved=sv1, x_low=x_low,
+               y_low=y_low)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
+    assert torch.equal(y_low, y1.to(torch.bfloat16))
+    assert torch.equal(H.saved_views(dw.cfg, sv1, dw.T)["xlow"], x_low)
+    dx0 = H.bwd(dw.cfg, lw, dw.x, dw.dy, sv0, dw.offsets, dw.timestamps, None)
+    lo = dw.dy.to(torch.bfloat16)
+    dx1 = H.bwd(dw.cfg, lw, dw.x, dw.dy, sv1, dw.offsets, dw.timestamps, None, dy_low=lo,
+                dx_low=lo)
+    torch.cuda.synchronize()
+    assert H.device_status() == 0
+    check_el(np_(dx1), np_(dx0).astype(np.float64), "bf16", "dX chained (aliased copies)")
+    assert torch.equal(lo, dx1.to(torch.bfloat16))
+
+
 def test_nvtx_ranges_leave_results_unchanged():
     """With NVTX ranges on (hstu_nvtx_enable), a stack forward gives the same
     bits as with them off; the ranges only mark the host timeline."""

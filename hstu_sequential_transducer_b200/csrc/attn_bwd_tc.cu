@@ -10,7 +10,9 @@
 // descending number of query tiles and dealt round-robin to one persistent
 // CTA per SM.  Per item the key tile's K and V stay in shared memory and the
 // CTA walks the query tiles that see it (causal: from the key tile on;
-// candidates see every history key):
+// candidates see every history key).  The head_dim-64 kernel, on 128-query
+// tiles (the head_dim-128 kernel further below walks 64-query blocks with
+// its own roles):
 //   warp 0      TMA producer: K, V once per item; Q_i, dO_i and the queries'
 //               timestamps per query tile
 //   warp 1      MMA issuer: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM; then
@@ -703,27 +705,26 @@ int sms();
 // A CTA owns one (key tile, head) item at a time and walks its query blocks
 // g = 0, 1, ... .  Per block the MMA thread computes S^T = K Q_g^T and
 // dP^T = V dO_g^T (128 keys x 64 queries, fp32 in TMEM); the activation warps
-// load both into registers, release the TMEM at once, and write P^T and dS
-// (bf16, [key][query] 128-byte swizzled tiles) to shared memory.  From there
-// the same tiles serve as the K-major A operand of dV += P^T dO and
-// dK += dS^T Q and as the MN-major B operand of dQ^T_g = K^T dS^T.  dQ^T has a
-// double buffer of its own in TMEM, so the next block's S^T, dP^T never wait
-// for the dQ drain: S^T(g+1) is issued as soon as block g's scores are in
-// registers.  A warpgroup of its own drains dQ^T(g) (transposes it into a
-// dense fp32 tile in shared memory and adds it to the fp32 dQ accumulator
-// with TMA bulk reduce-adds; rows past the sequence end carry exact zeros),
-// so the activation warps go from one block to the next without it; the
-// same warpgroup finishes an item with dK, dV times SiLU'(Pre) into dPre
-// while the activation warps already work on the next item, whose K and V
-// tiles the producer has prefetched into L2.  Off the fast path, a warp whose 32
-// columns hold no allowed pair writes zeros, and time gaps within +-2^31 s
-// take 32-bit bucket arithmetic.  Q/dO blocks come through a
-// three-stage ring that the producer keeps prefetched into L2, so block g+1's
-// loads overlap block g-1's dV/dK; the P^T and dS tiles are single-buffered
-// (block g is written once block g-1's MMAs have read them).  The layout packs
-// almost the whole 227 KB budget, so the kernel relies on a 1024-byte aligned
-// dynamic shared memory base (checked; it reports kStatusSmemAlign if not).
-// TMEM: S^T [0,64) dP^T [64,128) dQ^T_0 [128,192) dQ^T_1 [192,256)
+// load both into registers and release the TMEM at once, so S^T(g+1) can be
+// issued while they work.  They write P^T and dS^T (bf16 pairs) back into
+// TMEM, where they are the A operands of dV += P^T dO and dK += dS^T Q, and
+// dS ([key][query], a 128-byte swizzled tile) to shared memory, the
+// MN-major B operand of dQ^T_g = K^T dS^T.  A warpgroup of its own drains
+// dQ^T(g) from TMEM (transposes it into a dense fp32 tile in shared memory
+// and adds it to the fp32 dQ accumulator with TMA bulk reduce-adds; rows past
+// the sequence end carry exact zeros), so the activation warps go from one
+// block to the next without it; the same warpgroup finishes an item with dK,
+// dV times SiLU'(Pre) into dPre while the activation warps already work on
+// the next item, whose K and V tiles the producer has prefetched into L2.
+// Off the fast path, a warp whose 32 columns hold no allowed pair writes
+// zeros, and time gaps within +-2^31 s take 32-bit bucket arithmetic.  Q/dO
+// blocks come through a three-stage ring that the producer keeps prefetched
+// into L2, so block g+1's loads overlap block g-1's dV/dK; the P^T/dS^T
+// columns and the dS tile are single-buffered (block g writes them once block
+// g-1's MMAs have read them).  The layout packs almost the whole 227 KB
+// budget, so the kernel relies on a 1024-byte aligned dynamic shared memory
+// base (checked; it reports kStatusSmemAlign if not).
+// TMEM: S^T [0,64) dP^T [64,128) dQ^T [128,192) P^T [192,224) dS^T [224,256)
 //       dV [256,384) dK [384,512)
 constexpr int kQB = 64;
 constexpr int kQStages = 3;
